@@ -1,0 +1,265 @@
+"""ButterflyMoE expert-layer forward on NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of the C ABI in ``include/bfmoe.h`` (``libbfmoe.so``,
+built in-tree by ``python -m ternary_moe_butterfly_b200.build``).  The
+``bfmoe_*`` functions take raw pointers and sizes exactly like the C calls;
+the lower-case helpers take torch tensors and only marshal them (device
+pointers, the current CUDA stream, workspace sizing).  Every step of the
+layer runs in the library's CUDA kernels; there is no CPU or library
+fallback, and loading fails loudly if the shared library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbfmoe.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_NONFINITE, ERR_TIMEOUT, ERR_CUDA = range(7)
+F32, BF16 = 0, 1
+
+
+class BfmoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("status", "topk_idx", "gates", "perm", "offsets", "total")]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ternary_moe_butterfly_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "bfmoe_status_string": (ctypes.c_char_p, [I]),
+            "bfmoe_version": (I, []),
+            "bfmoe_packed_base_bytes": (Z, [I]),
+            "bfmoe_pack_base": (I, [P, I, ctypes.c_float, P, P]),
+            "bfmoe_route_workspace_bytes": (Z, [I, I, I]),
+            "bfmoe_route": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
+            "bfmoe_butterfly_workspace_bytes": (Z, [I, I]),
+            "bfmoe_butterfly_apply": (I, [P, I, I, I, I, P, P, I, P, P, Z, P]),
+            "bfmoe_forward_workspace_bytes": (Z, [I, I, I, I]),
+            "bfmoe_forward_ws_layout": (I, [I, I, I, I, ctypes.POINTER(WsLayout)]),
+            "bfmoe_forward": (I, [P, I, I, I, P, I, I, P, P, P, P, P, Z, P]),
+            "bfmoe_sync_status": (I, [P, P]),
+            "bfmoe_forward_profile": (I, [P, I, I, I, P, I, I, P, P, P, P, P, Z, P, P, P]),
+            "bfmoe_stage_name": (ctypes.c_char_p, [I]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ raw ABI
+# Same names and arguments as the C entry points (pointers as ints).
+
+def bfmoe_status_string(code):
+    return lib().bfmoe_status_string(int(code)).decode()
+
+
+status_string = bfmoe_status_string
+
+
+def bfmoe_version():
+    return lib().bfmoe_version()
+
+
+def bfmoe_packed_base_bytes(d):
+    return lib().bfmoe_packed_base_bytes(d)
+
+
+def bfmoe_pack_base(w, d, alpha, packed, stream):
+    return lib().bfmoe_pack_base(w, d, alpha, packed, stream)
+
+
+def bfmoe_route_workspace_bytes(T, N, k):
+    return lib().bfmoe_route_workspace_bytes(T, N, k)
+
+
+def bfmoe_route(logits, T, N, k, topk_idx, gates, perm, offsets, ws, ws_bytes, stream):
+    return lib().bfmoe_route(logits, T, N, k, topk_idx, gates, perm, offsets, ws, ws_bytes, stream)
+
+
+def bfmoe_butterfly_workspace_bytes(d, N):
+    return lib().bfmoe_butterfly_workspace_bytes(d, N)
+
+
+def bfmoe_butterfly_apply(x, dt, rows, d, N, angles, expert_of_row, transpose, y, ws, ws_bytes, stream):
+    return lib().bfmoe_butterfly_apply(x, dt, rows, d, N, angles, expert_of_row, transpose, y, ws, ws_bytes,
+                                       stream)
+
+
+def bfmoe_forward_workspace_bytes(T, d, N, k):
+    return lib().bfmoe_forward_workspace_bytes(T, d, N, k)
+
+
+def bfmoe_forward_ws_layout(T, d, N, k):
+    out = WsLayout()
+    code = lib().bfmoe_forward_ws_layout(T, d, N, k, ctypes.byref(out))
+    return code, out
+
+
+def bfmoe_forward(x, dt, T, d, logits, N, k, packed_base, theta, phi, y, ws, ws_bytes, stream):
+    return lib().bfmoe_forward(x, dt, T, d, logits, N, k, packed_base, theta, phi, y, ws, ws_bytes, stream)
+
+
+def bfmoe_sync_status(ws, stream):
+    return lib().bfmoe_sync_status(ws, stream)
+
+
+MAX_STAGES = 16
+
+
+def bfmoe_forward_profile(x, dt, T, d, logits, N, k, packed_base, theta, phi, y, ws, ws_bytes, stream, stage_ms,
+                          n_stages):
+    return lib().bfmoe_forward_profile(x, dt, T, d, logits, N, k, packed_base, theta, phi, y, ws, ws_bytes, stream,
+                                       stage_ms, n_stages)
+
+
+def bfmoe_stage_name(i):
+    r = lib().bfmoe_stage_name(int(i))
+    return None if r is None else r.decode()
+
+
+# ------------------------------------------------------- tensor marshalling
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream=None):
+    if stream is not None:
+        return int(getattr(stream, "cuda_stream", stream))
+    return int(_torch().cuda.current_stream().cuda_stream)
+
+
+def _dt(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"x must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else int(t.data_ptr())
+
+
+def _check(code, what):
+    if code != OK:
+        raise BfmoeError(code, what)
+
+
+def _ws(nbytes, device):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def pack_base(w, alpha: float, stream=None):
+    """int8 [d][d] ternary (device) -> packed uint8 tensor (synchronises)."""
+    torch = _torch()
+    d = int(w.shape[0])
+    out = torch.empty(max(int(bfmoe_packed_base_bytes(d)), 16), dtype=torch.uint8, device=w.device)
+    _check(bfmoe_pack_base(_ptr(w.contiguous()), d, float(alpha), _ptr(out), _stream(stream)), "bfmoe_pack_base")
+    return out
+
+
+def route(logits, k: int, ws=None, stream=None):
+    """Top-k routing and bucketing; returns (topk_idx, gates, perm, offsets, ws)."""
+    torch = _torch()
+    T, N = map(int, logits.shape)
+    dev = logits.device
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    need = bfmoe_route_workspace_bytes(T, N, k)
+    if ws is None:
+        ws = _ws(need, dev)
+    _check(bfmoe_route(_ptr(logits), T, N, k, _ptr(idx), _ptr(gates), _ptr(perm), _ptr(offsets), _ptr(ws),
+                       ws.numel(), _stream(stream)), "bfmoe_route")
+    return idx, gates, perm, offsets, ws
+
+
+def butterfly_apply(x, angles, expert_of_row=None, transpose: bool = False, ws=None, out=None, stream=None):
+    """y[r] = B(angles[e_r]) x[r] (or B^T); x [rows][d] fp32/bf16 on the device."""
+    torch = _torch()
+    rows, d = map(int, x.shape)
+    N = int(angles.shape[0])
+    y = torch.empty_like(x) if out is None else out
+    if ws is None:
+        ws = _ws(bfmoe_butterfly_workspace_bytes(d, N), x.device)
+    _check(bfmoe_butterfly_apply(_ptr(x), _dt(x), rows, d, N, _ptr(angles), _ptr(expert_of_row),
+                                 int(bool(transpose)), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
+           "bfmoe_butterfly_apply")
+    return y, ws
+
+
+def forward_workspace(T: int, d: int, N: int, k: int, device):
+    return _ws(bfmoe_forward_workspace_bytes(T, d, N, k), device)
+
+
+def forward(x, logits, k: int, packed, theta, phi, ws=None, out=None, stream=None):
+    """The expert layer: y = sum_j g_j alpha B(phi_e) W_base B(theta_e)^T x."""
+    torch = _torch()
+    T, d = map(int, x.shape)
+    N = int(logits.shape[1])
+    y = torch.empty_like(x) if out is None else out
+    if ws is None:
+        ws = forward_workspace(T, d, N, k, x.device)
+    _check(bfmoe_forward(_ptr(x), _dt(x), T, d, _ptr(logits), N, k, _ptr(packed), _ptr(theta), _ptr(phi), _ptr(y),
+                         _ptr(ws), ws.numel(), _stream(stream)), "bfmoe_forward")
+    return y, ws
+
+
+def forward_routing(ws, T: int, d: int, N: int, k: int):
+    """Views of the routing results bfmoe_forward left in its workspace:
+    (topk_idx [T][k], gates [T][k], perm [T*k], offsets [N+1])."""
+    torch = _torch()
+    code, lay = bfmoe_forward_ws_layout(T, d, N, k)
+    _check(code, "bfmoe_forward_ws_layout")
+
+    def view(off, n, dtype):
+        return ws[off:off + 4 * n].view(dtype)
+
+    idx = view(lay.topk_idx, T * k, torch.int32).view(T, k)
+    gates = view(lay.gates, T * k, torch.float32).view(T, k)
+    perm = view(lay.perm, T * k, torch.int32)
+    offsets = view(lay.offsets, N + 1, torch.int32)
+    return idx, gates, perm, offsets
+
+
+def forward_profile(x, logits, k: int, packed, theta, phi, ws, out, stream=None):
+    """bfmoe_forward with a CUDA event after each kernel (synchronises);
+    returns {stage name: milliseconds}."""
+    T, d = map(int, x.shape)
+    N = int(logits.shape[1])
+    ms = (ctypes.c_float * MAX_STAGES)()
+    n = ctypes.c_int(0)
+    _check(bfmoe_forward_profile(_ptr(x), _dt(x), T, d, _ptr(logits), N, k, _ptr(packed), _ptr(theta), _ptr(phi),
+                                 _ptr(out), _ptr(ws), ws.numel(), _stream(stream),
+                                 ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(ctypes.pointer(n), ctypes.c_void_p)),
+           "bfmoe_forward_profile")
+    return {bfmoe_stage_name(i): float(ms[i]) for i in range(n.value)}
+
+
+def sync_status(ws, stream=None) -> int:
+    """Synchronise and return (and clear) the device status word of ws."""
+    return int(bfmoe_sync_status(_ptr(ws), _stream(stream)))
