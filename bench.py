@@ -134,7 +134,7 @@ def cpu_oracle_rate(w: wl.Workload, target_s: float, inp=None, max_tokens=None):
     t0 = time.perf_counter()
     oracle.forward(inp.x[:n], inp.logits[:n], w.k, inp.w_base, inp.alpha, inp.theta, inp.phi)
     per_tok = max((time.perf_counter() - t0) / n, 1e-6)
-    n2 = int(max(n, min(inp.x.shape[0] if max_tokens is None else max_tokens, target_s / per_tok)))
+    n2 = int(max(n, min(1 << 20 if max_tokens is None else max_tokens, target_s / per_tok)))
     reps = max(1, int(math.ceil(n2 / inp.x.shape[0])))
     xs = np.concatenate([inp.x] * reps)[:n2]
     ls = np.concatenate([inp.logits] * reps)[:n2]
@@ -220,42 +220,47 @@ def run_ours(args, w):
         bf.forward(xs[s], ls[s], k, packed, theta, phi, ws=ws, out=ys[s], stream=stream)
 
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
+        for i in range(args.warmup):
             step(i % nsets)
     st = bf.sync_status(ws, stream)
     if st != bf.OK:
         raise RuntimeError(f"warm-up status {bf.status_string(st)}")
 
-    # one graph holds one step per input set
+    # exactly K timed steps, cycling through the input sets, in one graph
+    K = args.steps
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
-            for s in range(nsets):
-                step(s)
-    reps = max(1, int(math.ceil(args.steps / nsets)))
-    ksteps = reps * nsets
-    with torch.cuda.stream(stream):
+            for i in range(K):
+                step(i % nsets)
         graph.replay()
     stream.synchronize()
 
+    # clocks: sample through a soak of back-to-back replays and the timed
+    # region that follows it
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_id = vis.split(",")[local].strip() if vis else str(device.index)
     sampler = ClockSampler(smi_id)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        t_end = time.perf_counter() + args.soak_seconds
+        while time.perf_counter() < t_end:
+            graph.replay()
+            stream.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
+    with torch.cuda.stream(stream):
+        e0.record(stream)
         graph.replay()
-    e1.record(stream)
+        e1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1) / ksteps
+    ms = e0.elapsed_time(e1) / K
+    ksteps = K
     st = bf.sync_status(ws, stream)
     if st != bf.OK:
         raise RuntimeError(f"timed status {bf.status_string(st)}")
@@ -266,7 +271,7 @@ def run_ours(args, w):
 
     # per-kernel durations (events between the launches of one step)
     prof = {}
-    nprof = min(50, max(10, args.steps))
+    nprof = args.profile_steps
     with torch.cuda.stream(stream):
         for i in range(nprof):
             r = bf.forward_profile(xs[i % nsets], ls[i % nsets], k, packed, theta, phi, ws, ys[i % nsets],
@@ -289,25 +294,25 @@ def run_ours(args, w):
         hy[s].copy_(dy, non_blocking=True)
 
     with torch.cuda.stream(stream):
-        for i in range(3):
+        for i in range(max(args.warmup, 1)):
             e2e_step(i % nsets)
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g2, stream=stream):
-            for s in range(nsets):
-                e2e_step(s)
+            for i in range(K):
+                e2e_step(i % nsets)
         g2.replay()
     stream.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(reps):
+    with torch.cuda.stream(stream):
+        f0.record(stream)
         g2.replay()
-    f1.record(stream)
+        f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / ksteps
+    e2e_ms = f0.elapsed_time(f1) / K
     if world > 1:
         t = torch.tensor([e2e_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -351,7 +356,7 @@ def run_ours(args, w):
     if rank == 0:
         line = {
             "metric": "ButterflyMoE layer routed tokens/s (d=%d,N=%d,top-%d)" % (d, N, k),
-            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": ksteps, "warmup": max(args.warmup, 3),
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": ksteps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "d": d, "N": N, "k": k, "T": T, "x": w.dtype,
@@ -383,9 +388,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--profile-steps", type=int, default=20)
     ap.add_argument("--config", default="headline", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--soak-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.config]

@@ -42,7 +42,7 @@ def to_x(inp):
 
 
 def check_close(y, ref, what=""):
-    y = y.double()
+    y = np.asarray(y, dtype=np.float64)
     fro = np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300)
     mx = np.abs(y - ref).max() / max(np.abs(ref).max(), 1e-300)
     assert fro <= REL_FRO and mx <= REL_MAX, f"{what}: rel fro {fro:.3e}, rel max {mx:.3e}"
