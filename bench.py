@@ -328,10 +328,14 @@ def run_ours(args, w):
 
     # dominant kernel and its roofline
     R, Rp, L = T * k, (T * k + 127) // 128 * 128, w.L
+    rot = R * L * (d // 2)  # Givens rotations per butterfly pass over all rows
+    sm_mhz = (clocks or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    alu_peak = 148 * 128 * sm_mhz * 1e6 / 1e12  # FP32 lane-instructions, Tops/s
     models = {
         "contract": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
-        "expert_in": ("hbm", R * d * xb + Rp * d * 2 + T * k * 8, "GB/s"),
-        "expert_out": ("hbm", Rp * d * 4 + T * d * xb + T * k * 12, "GB/s"),
+        "expert_in": ("alu", 4.0 * rot, "Tops/s"),
+        "combine": ("hbm", R * d * 4 + T * d * xb + T * k * 8, "GB/s"),
+        "route": ("hbm", T * N * 4 + T * k * 12, "GB/s"),
     }
     dom = max(prof, key=prof.get) if prof else None
     roof = None
@@ -341,6 +345,9 @@ def run_ours(args, w):
         if bound == "tensor":
             achieved = amount / sec / 1e12
             peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        elif bound == "alu":
+            achieved = amount / sec / 1e12
+            peak = alu_peak
         else:
             achieved = amount / sec / 1e9
             peak = peaks["hbm_gbs"]

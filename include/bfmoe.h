@@ -188,6 +188,14 @@ BFMOE_API bfmoe_status bfmoe_forward_profile(const void *x, bfmoe_dtype dt, int 
  * out of range). */
 BFMOE_API const char *bfmoe_stage_name(int i);
 
+/* Test hooks (process-wide, not for production use).
+ * BFMOE_DEBUG_SKIP_ARRIVE_BLOCK: the routing block with this index returns
+ * before its first grid barrier (-1, the default, disables the hook), so
+ * the other blocks' bounded waits run out and the call reports
+ * BFMOE_ERR_TIMEOUT through the status word instead of hanging. */
+#define BFMOE_DEBUG_SKIP_ARRIVE_BLOCK 1
+BFMOE_API void bfmoe_debug_set(int key, int value);
+
 /* Synchronise `stream`, then return (and clear) the status word at the start
  * of `ws` (a route, butterfly or forward workspace). */
 BFMOE_API bfmoe_status bfmoe_sync_status(void *ws, void *stream);

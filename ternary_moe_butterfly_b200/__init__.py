@@ -56,6 +56,7 @@ def lib():
             "bfmoe_sync_status": (I, [P, P]),
             "bfmoe_forward_profile": (I, [P, I, I, I, P, I, I, P, P, P, P, P, Z, P, P, P]),
             "bfmoe_stage_name": (ctypes.c_char_p, [I]),
+            "bfmoe_debug_set": (None, [I, I]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -129,6 +130,14 @@ def bfmoe_forward_profile(x, dt, T, d, logits, N, k, packed_base, theta, phi, y,
                           n_stages):
     return lib().bfmoe_forward_profile(x, dt, T, d, logits, N, k, packed_base, theta, phi, y, ws, ws_bytes, stream,
                                        stage_ms, n_stages)
+
+
+DEBUG_SKIP_ARRIVE_BLOCK = 1
+
+
+def bfmoe_debug_set(key, value):
+    """Test hook; see include/bfmoe.h."""
+    lib().bfmoe_debug_set(int(key), int(value))
 
 
 def bfmoe_stage_name(i):

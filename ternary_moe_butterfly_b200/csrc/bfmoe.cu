@@ -8,6 +8,9 @@
 #include <mutex>
 #include <utility>
 
+#include <algorithm>
+
+#include "contract.cuh"
 #include "layer.cuh"
 #include "route.cuh"
 
@@ -49,10 +52,12 @@ bfmoe_status check_route_shape(int T, int N, int k)
     return BFMOE_OK;
 }
 
-int route_blocks(int T) { return (T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock; }
+int route_chunks(int T) { return (T + kRouteChunk - 1) / kRouteChunk; }
 
+// Status word and grid-barrier counter share the first 16 bytes of every
+// workspace; one memset clears both.
 struct RouteLayout {
-    size_t status, hist, total;
+    size_t status, hist, total, total_bytes;
 };
 
 RouteLayout route_layout(int T, int N)
@@ -62,16 +67,20 @@ RouteLayout route_layout(int T, int N)
     l.status = o;
     o += kAlign;
     l.hist = o;
-    o += align_up((size_t)route_blocks(T) * N * 4);
+    o += align_up((size_t)route_chunks(T) * N * 4);
     l.total = o;
+    o += align_up((size_t)N * 4);
+    l.total_bytes = o;
     return l;
 }
 
 struct FwdLayout {
-    size_t status, topk_idx, gates, perm, row_pos, offsets, hist, coef_t, coef_p, wdec, a_blocks, z, total;
+    size_t status, topk_idx, gates, perm, offsets, hist, total, tiles, ntiles, coef_t, coef_p, wdec, a_blocks,
+        slot, total_bytes;
 };
 
 int padded_rows(int T, int k) { return (T * k + kBM - 1) / kBM * kBM; }
+int max_in_tiles(int T, int d, int N, int k) { return (T * k + tile_rows_for(d) - 1) / tile_rows_for(d) + N; }
 
 FwdLayout fwd_layout(int T, int d, int N, int k)
 {
@@ -88,61 +97,78 @@ FwdLayout fwd_layout(int T, int d, int N, int k)
     l.topk_idx = take(R * 4);
     l.gates = take(R * 4);
     l.perm = take(R * 4);
-    l.row_pos = take(R * 4);
     l.offsets = take(((size_t)N + 1) * 4);
-    l.hist = take((size_t)route_blocks(T) * N * 4);
+    l.hist = take((size_t)route_chunks(T) * N * 4);
+    l.total = take((size_t)N * 4);
+    l.tiles = take((size_t)max_in_tiles(T, d, N, k) * 16);
+    l.ntiles = take(4);
     l.coef_t = take(ncoef * 8);
     l.coef_p = take(ncoef * 8);
     l.wdec = take((size_t)d * d * 2);
     l.a_blocks = take(Rp * d * 2);
-    l.z = take(Rp * d * 4);
-    l.total = o;
+    l.slot = take(R * d * 4);
+    l.total_bytes = o;
     return l;
+}
+
+// Per-device facts and per-(device, kernel, smem) attributes, cached.
+std::mutex g_mu;
+std::map<std::pair<int, const void *>, size_t> g_smem_attr;
+std::map<std::pair<std::pair<int, const void *>, size_t>, int> g_occ;
+std::map<int, int> g_sms;
+
+int device_sms()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> g(g_mu);
+    auto it = g_sms.find(dev);
+    if (it != g_sms.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    g_sms[dev] = n;
+    return n;
 }
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per
 // (device, kernel, size).
-std::mutex g_attr_mu;
-std::map<std::pair<int, const void *>, size_t> g_attr;
-
 bool ensure_smem(const void *fn, size_t bytes)
 {
     if (bytes <= 48 * 1024) return true;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    std::lock_guard<std::mutex> g(g_attr_mu);
+    std::lock_guard<std::mutex> g(g_mu);
     auto key = std::make_pair(dev, fn);
-    auto it = g_attr.find(key);
-    if (it != g_attr.end() && it->second >= bytes) return true;
+    auto it = g_smem_attr.find(key);
+    if (it != g_smem_attr.end() && it->second >= bytes) return true;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
-    g_attr[key] = bytes;
+    g_smem_attr[key] = bytes;
     return true;
 }
 
-bfmoe_status launched()
+// Resident blocks per SM of `fn` at `threads` x `smem` (0 on failure).
+int occupancy(const void *fn, int threads, size_t smem)
 {
-    return cudaGetLastError() == cudaSuccess ? BFMOE_OK : BFMOE_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    {
+        std::lock_guard<std::mutex> g(g_mu);
+        auto it = g_occ.find(std::make_pair(std::make_pair(dev, fn), smem));
+        if (it != g_occ.end()) return it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> g(g_mu);
+    g_occ[std::make_pair(std::make_pair(dev, fn), smem)] = n;
+    return n;
 }
 
-// Routing launches shared by bfmoe_route and bfmoe_forward.
-struct StageRec;
-void mark(StageRec *r, cudaStream_t st);
+bfmoe_status launched() { return cudaGetLastError() == cudaSuccess ? BFMOE_OK : BFMOE_ERR_CUDA; }
 
-bfmoe_status launch_route(const float *logits, int T, int N, int k, int32_t *idx, float *gates, int32_t *perm,
-                          int32_t *offsets, int32_t *row_pos, int32_t *hist, uint32_t *status, cudaStream_t st,
-                          StageRec *rec = nullptr)
-{
-    const int nblk = route_blocks(T);
-    if (!ensure_smem((const void *)k_bucket_scan, (size_t)(N + 1024) * 4)) return BFMOE_ERR_CUDA;
-    k_topk<<<nblk, kRouteThreads, (size_t)N * 4, st>>>(logits, T, N, k, idx, gates, hist, status);
-    mark(rec, st);
-    k_bucket_scan<<<1, 1024, (size_t)(N + 1024) * 4, st>>>(hist, nblk, N, offsets);
-    mark(rec, st);
-    k_bucket_scatter<<<nblk, kRouteThreads, (size_t)N * 4, st>>>(idx, hist, T, N, k, perm, row_pos);
-    mark(rec, st);
-    return launched();
-}
+// Process-wide test hook (bfmoe_debug_set): the routing block that skips the
+// first grid barrier, or -1.
+int g_skip_arrive_block = -1;
 
 // Optional per-kernel event recorder used by bfmoe_forward_profile.
 struct StageRec {
@@ -151,19 +177,61 @@ struct StageRec {
     bool on = false;
 };
 
-const char *const kStageNames[] = {"coef", "decode_base", "route_topk", "route_scan", "route_scatter",
-                                   "expert_in", "contract", "expert_out"};
-constexpr int kNumStages = 8;
+const char *const kStageNames[] = {"route", "expert_in", "contract", "combine"};
+constexpr int kNumStages = 4;
 
 void mark(StageRec *r, cudaStream_t st)
 {
     if (r && r->on && r->n <= BFMOE_MAX_STAGES) cudaEventRecord(r->ev[r->n++], st);
 }
 
+template <typename K, typename... Args>
+cudaError_t launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, bool coop,
+                   Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (coop) {
+        attr[na].id = cudaLaunchAttributeCooperative;
+        attr[na].val.cooperative = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// The routing kernel, launched cooperatively on as many blocks as fit.
+bfmoe_status launch_route(RouteParams rp, cudaStream_t st)
+{
+    const size_t smem = route_smem_bytes(rp.N);
+    if (!ensure_smem((const void *)k_route, smem)) return BFMOE_ERR_CUDA;
+    const int sms = device_sms();
+    const int occ = occupancy((const void *)k_route, kRouteThreads, smem);
+    if (sms <= 0 || occ <= 0) return BFMOE_ERR_CUDA;
+    const int nchunk = route_chunks(rp.T);
+    int grid = std::max(nchunk, 2 * sms);
+    grid = std::min(grid, occ * sms);
+    rp.skip_arrive_block = g_skip_arrive_block;
+    if (launch(k_route, dim3(grid), dim3(kRouteThreads), smem, st, false, true, rp) != cudaSuccess)
+        return BFMOE_ERR_CUDA;
+    return BFMOE_OK;
+}
+
 template <typename T>
 bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void *packed, const float *theta,
                           const float *phi, void *y, uint8_t *ws, const FwdLayout &l, const float *logits,
-                          cudaStream_t st, StageRec *rec = nullptr)
+                          cudaStream_t st, StageRec *rec)
 {
     const int L = ilog2(d);
     const int R = T_ * k, Rp = padded_rows(T_, k);
@@ -171,46 +239,121 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     int32_t *idx = reinterpret_cast<int32_t *>(ws + l.topk_idx);
     float *gates = reinterpret_cast<float *>(ws + l.gates);
     int32_t *perm = reinterpret_cast<int32_t *>(ws + l.perm);
-    int32_t *row_pos = reinterpret_cast<int32_t *>(ws + l.row_pos);
-    int32_t *offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
-    int32_t *hist = reinterpret_cast<int32_t *>(ws + l.hist);
     float2 *ct = reinterpret_cast<float2 *>(ws + l.coef_t);
     float2 *cp = reinterpret_cast<float2 *>(ws + l.coef_p);
     __half *wdec = reinterpret_cast<__half *>(ws + l.wdec);
     __half *ablk = reinterpret_cast<__half *>(ws + l.a_blocks);
-    float *z = reinterpret_cast<float *>(ws + l.z);
+    float *slot = reinterpret_cast<float *>(ws + l.slot);
+    int4 *tiles = reinterpret_cast<int4 *>(ws + l.tiles);
+    int32_t *ntiles = reinterpret_cast<int32_t *>(ws + l.ntiles);
+    const int sms = device_sms();
+    if (sms <= 0) return BFMOE_ERR_CUDA;
 
-    if (cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return BFMOE_ERR_CUDA;
+    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);
-    const int ncoef = N * L * (d / 2);
-    k_coef<<<(2 * ncoef + 255) / 256, 256, 0, st>>>(theta, phi, ncoef, ct, cp);
-    mark(rec, st);
-    const size_t nchunks = (size_t)d * d / 8;
-    k_decode_base<<<(unsigned)((nchunks + 255) / 256), 256, 0, st>>>(reinterpret_cast<const uint32_t *>(packed), d,
-                                                                       wdec, status);
-    mark(rec, st);
-    bfmoe_status s = launch_route(logits, T_, N, k, idx, gates, perm, offsets, row_pos, hist, status, st, rec);
+
+    RouteParams rp{};
+    rp.logits = logits;
+    rp.T = T_;
+    rp.N = N;
+    rp.k = k;
+    rp.topk_idx = idx;
+    rp.gates = gates;
+    rp.perm = perm;
+    rp.row_pos = nullptr;
+    rp.offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
+    rp.hist = reinterpret_cast<int32_t *>(ws + l.hist);
+    rp.total = reinterpret_cast<int32_t *>(ws + l.total);
+    rp.sync = status + 1;
+    rp.status = status;
+    rp.theta = theta;
+    rp.phi = phi;
+    rp.coef_t = ct;
+    rp.coef_p = cp;
+    rp.ncoef = N * L * (d / 2);
+    rp.packed = reinterpret_cast<const uint32_t *>(packed);
+    rp.wdec = wdec;
+    rp.d = d;
+    rp.in_tiles = tiles;
+    rp.n_in_tiles = ntiles;
+    rp.tile_rows = tile_rows_for(d);
+    bfmoe_status s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
-
-    const int RT = tile_rows_for(d);
-    const size_t in_smem = rows_smem_bytes(d, 2);
-    if (!ensure_smem((const void *)k_expert_in<T>, in_smem)) return BFMOE_ERR_CUDA;
-    k_expert_in<T><<<Rp / RT, 256, in_smem, st>>>(reinterpret_cast<const T *>(x), d, L, k, R, perm, idx, ct, ablk,
-                                                  status);
     mark(rec, st);
 
+    ExpertInParams ep{};
+    ep.x = x;
+    ep.d = d;
+    ep.L = L;
+    ep.k = k;
+    ep.N = N;
+    ep.R = R;
+    ep.perm = perm;
+    ep.tiles = tiles;
+    ep.n_tiles = ntiles;
+    ep.max_tiles = max_in_tiles(T_, d, N, k);
+    ep.coef_t = ct;
+    ep.a_blocks = ablk;
+    ep.status = status;
+    const bool smc = expert_in_smem_coef(d, L);
+    const size_t in_smem = expert_in_smem_bytes(d, L, smc);
+    auto kin = smc ? k_expert_in<T, true> : k_expert_in<T, false>;
+    if (!ensure_smem((const void *)kin, in_smem)) return BFMOE_ERR_CUDA;
+    const int in_occ = occupancy((const void *)kin, 256, in_smem);
+    const int in_grid = std::max(1, std::min(max_in_tiles(T_, d, N, k), std::max(1, in_occ) * sms));
+    if (launch(kin, dim3(in_grid), dim3(256), in_smem, st, true, false, ep) != cudaSuccess) return BFMOE_ERR_CUDA;
+    mark(rec, st);
+
+    ContractParams cpar{};
+    cpar.a_blocks = ablk;
+    cpar.w_blocks = wdec;
+    cpar.slot = slot;
+    cpar.perm = perm;
+    cpar.topk_idx = idx;
+    cpar.coef_p = cp;
+    cpar.d = d;
+    cpar.L = L;
+    cpar.N = N;
+    cpar.R = R;
+    cpar.Rp = Rp;
+    cpar.status = status;
+    const int BN = gemm_bn(d);
+    const int nunits = (Rp / kBM) * (d / BN);
     const size_t c_smem = contract_smem_bytes(d);
-    if (!ensure_smem((const void *)k_contract, c_smem)) return BFMOE_ERR_CUDA;
-    dim3 cgrid(Rp / kBM, d / gemm_bn(d));
-    k_contract<<<cgrid, 128, c_smem, st>>>(ablk, wdec, z, d, status);
+    auto kc = BN == 256 ? k_contract<256> : (BN == 128 ? k_contract<128> : k_contract<64>);
+    if (!ensure_smem((const void *)kc, c_smem)) return BFMOE_ERR_CUDA;
+    if (launch(kc, dim3(std::min(nunits, sms)), dim3(kContractThreads), c_smem, st, true, false, cpar) !=
+        cudaSuccess)
+        return BFMOE_ERR_CUDA;
     mark(rec, st);
 
-    const int TT = RT / k > 0 ? RT / k : 1;
-    const size_t out_smem = (size_t)TT * k * (d + 1) * 4 + (size_t)TT * k * 12;
-    if (!ensure_smem((const void *)k_expert_out<T>, out_smem)) return BFMOE_ERR_CUDA;
-    k_expert_out<T><<<(T_ + TT - 1) / TT, 256, out_smem, st>>>(z, d, L, T_, k, row_pos, idx, gates, cp,
-                                                              reinterpret_cast<const uint32_t *>(packed),
-                                                              reinterpret_cast<T *>(y));
+    CombineParams cb{};
+    cb.slot = slot;
+    cb.T = T_;
+    cb.d = d;
+    cb.L = L;
+    cb.k = k;
+    cb.N = N;
+    cb.s_lo = ilog2(BN);
+    cb.topk_idx = idx;
+    cb.gates = gates;
+    cb.coef_p = cp;
+    cb.packed = reinterpret_cast<const uint32_t *>(packed);
+    cb.y = y;
+    const int HS = L - cb.s_lo;
+    cudaError_t e = cudaSuccess;
+    switch (HS) {
+    case 0: {
+        const size_t nthreads = (size_t)T_ * (d / 8);
+        e = launch(k_combine_sum<T>, dim3((unsigned)((nthreads + 255) / 256)), dim3(256), 0, st, true, false, cb);
+        break;
+    }
+    case 1: e = launch(k_combine_high<T, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    case 2: e = launch(k_combine_high<T, 2>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    case 3: e = launch(k_combine_high<T, 3>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    default: e = launch(k_combine_high<T, 4>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    }
+    if (e != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);
     return launched();
 }
@@ -269,7 +412,7 @@ bfmoe_status bfmoe_pack_base(const int8_t *w, int d, float alpha, void *packed, 
 size_t bfmoe_route_workspace_bytes(int T, int N, int k)
 {
     if (check_route_shape(T, N, k) != BFMOE_OK) return 0;
-    return route_layout(T, N).total;
+    return route_layout(T, N).total_bytes;
 }
 
 bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk_idx, float *gates, int32_t *perm,
@@ -282,13 +425,32 @@ bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk
         !aligned(perm, 4) || !aligned(offsets, 4))
         return BFMOE_ERR_INVALID_ARG;
     const RouteLayout l = route_layout(T, N);
-    if (ws_bytes < l.total) return BFMOE_ERR_WORKSPACE;
+    if (ws_bytes < l.total_bytes) return BFMOE_ERR_WORKSPACE;
     uint8_t *w = reinterpret_cast<uint8_t *>(ws);
     cudaStream_t st = as_stream(stream);
     uint32_t *status = reinterpret_cast<uint32_t *>(w + l.status);
-    if (cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return BFMOE_ERR_CUDA;
-    return launch_route(logits, T, N, k, topk_idx, gates, perm, offsets, nullptr,
-                        reinterpret_cast<int32_t *>(w + l.hist), status, st);
+    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
+    RouteParams rp{};
+    rp.logits = logits;
+    rp.T = T;
+    rp.N = N;
+    rp.k = k;
+    rp.topk_idx = topk_idx;
+    rp.gates = gates;
+    rp.perm = perm;
+    rp.offsets = offsets;
+    rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
+    rp.total = reinterpret_cast<int32_t *>(w + l.total);
+    rp.sync = status + 1;
+    rp.status = status;
+    s = launch_route(rp, st);
+    if (s != BFMOE_OK) return s;
+    return launched();
+}
+
+void bfmoe_debug_set(int key, int value)
+{
+    if (key == BFMOE_DEBUG_SKIP_ARRIVE_BLOCK) g_skip_arrive_block = value;
 }
 
 size_t bfmoe_butterfly_workspace_bytes(int d, int N)
@@ -320,7 +482,7 @@ bfmoe_status bfmoe_butterfly_apply(const void *x, bfmoe_dtype dt, int rows, int 
     if (rows == 0) return BFMOE_OK;
     const int L = ilog2(d);
     const int ncoef = N * L * (d / 2);
-    k_coef<<<(ncoef + 255) / 256, 256, 0, st>>>(angles, nullptr, ncoef, coef, nullptr);
+    k_coef<<<(ncoef + 255) / 256, 256, 0, st>>>(angles, ncoef, coef);
     const int RT = tile_rows_for(d);
     const size_t smem = rows_smem_bytes(d, 1);
     const unsigned grid = (unsigned)((rows + RT - 1) / RT);
@@ -340,7 +502,7 @@ bfmoe_status bfmoe_butterfly_apply(const void *x, bfmoe_dtype dt, int rows, int 
 size_t bfmoe_forward_workspace_bytes(int T, int d, int N, int k)
 {
     if (check_d(d) != BFMOE_OK || check_route_shape(T, N, k) != BFMOE_OK) return 0;
-    return fwd_layout(T, d, N, k).total;
+    return fwd_layout(T, d, N, k).total_bytes;
 }
 
 bfmoe_status bfmoe_forward_ws_layout(int T, int d, int N, int k, bfmoe_ws_layout *out)
@@ -356,7 +518,7 @@ bfmoe_status bfmoe_forward_ws_layout(int T, int d, int N, int k, bfmoe_ws_layout
     out->gates = l.gates;
     out->perm = l.perm;
     out->offsets = l.offsets;
-    out->total = l.total;
+    out->total = l.total_bytes;
     return BFMOE_OK;
 }
 
@@ -375,7 +537,7 @@ static bfmoe_status forward_impl(const void *x, bfmoe_dtype dt, int T, int d, co
         return BFMOE_ERR_INVALID_ARG;
     if (x == y) return BFMOE_ERR_INVALID_ARG;
     const FwdLayout l = fwd_layout(T, d, N, k);
-    if (ws_bytes < l.total) return BFMOE_ERR_WORKSPACE;
+    if (ws_bytes < l.total_bytes) return BFMOE_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);
     uint8_t *w = reinterpret_cast<uint8_t *>(ws);
     if (dt == BFMOE_F32) return launch_layer<float>(x, T, d, N, k, packed_base, theta, phi, y, w, l, logits, st, rec);

@@ -41,7 +41,7 @@ __device__ __forceinline__ void bfly_subset(float *row, int base, int s0, const 
             if (m & (1 << ls)) continue;
             const int j = base + (m << s0);
             const int p = ((j >> (s + 1)) << s) | (j & (h - 1));
-            const float2 c = __ldg(cs + p);
+            const float2 c = cs[p];
             const float sn = TRANSPOSE ? -c.y : c.y;
             const float a = v[m], b = v[m + (1 << ls)];
             v[m] = fmaf(c.x, a, -(sn * b));
@@ -52,9 +52,11 @@ __device__ __forceinline__ void bfly_subset(float *row, int base, int s0, const 
     for (int m = 0; m < M; ++m) row[base + (m << s0)] = v[m];
 }
 
+// Row r uses the table  coef + sexp[r] * estride  (sexp == nullptr: every
+// row uses `coef`, e.g. one expert's table staged in shared memory).
 template <int G, bool TRANSPOSE>
-__device__ void bfly_pass(float *tile, int ld, int rows, int d, int L, int s0, const int *sexp,
-                          const float2 *__restrict__ coef, int nthreads)
+__device__ void bfly_pass(float *tile, int ld, int rows, int d, int s0, const int *sexp,
+                          const float2 *__restrict__ coef, size_t estride, int nthreads)
 {
     const int half = d >> 1;
     const int nsub = d >> G;
@@ -64,39 +66,41 @@ __device__ void bfly_pass(float *tile, int ld, int rows, int d, int L, int s0, c
         const int r = it % rows;
         const int sub = it / rows;
         const int base = ((sub >> s0) << s1) | (sub & ((1 << s0) - 1));
-        const float2 *cf = coef + (size_t)sexp[r] * L * half;
+        const float2 *cf = sexp ? coef + (size_t)sexp[r] * estride : coef;
         bfly_subset<G, TRANSPOSE>(tile + (size_t)r * ld, base, s0, cf, half);
     }
 }
 
 template <bool TRANSPOSE>
-__device__ __forceinline__ void bfly_pass_g(int g, float *tile, int ld, int rows, int d, int L, int s0,
-                                            const int *sexp, const float2 *coef, int nthreads)
+__device__ __forceinline__ void bfly_pass_g(int g, float *tile, int ld, int rows, int d, int s0, const int *sexp,
+                                            const float2 *coef, size_t estride, int nthreads)
 {
     switch (g) {
-    case 1: bfly_pass<1, TRANSPOSE>(tile, ld, rows, d, L, s0, sexp, coef, nthreads); break;
-    case 2: bfly_pass<2, TRANSPOSE>(tile, ld, rows, d, L, s0, sexp, coef, nthreads); break;
-    case 3: bfly_pass<3, TRANSPOSE>(tile, ld, rows, d, L, s0, sexp, coef, nthreads); break;
-    case 4: bfly_pass<4, TRANSPOSE>(tile, ld, rows, d, L, s0, sexp, coef, nthreads); break;
-    default: bfly_pass<5, TRANSPOSE>(tile, ld, rows, d, L, s0, sexp, coef, nthreads); break;
+    case 1: bfly_pass<1, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
+    case 2: bfly_pass<2, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
+    case 3: bfly_pass<3, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
+    case 4: bfly_pass<4, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
+    default: bfly_pass<5, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
     }
 }
 
-// Apply B (transpose == false) or B^T (transpose == true) of expert sexp[r]
-// to every row r < rows of the tile.  Must be called by all threads of the
-// block (contains __syncthreads).
+// Apply B (transpose == false) or B^T (transpose == true) to every row r <
+// rows of the tile; row r uses the table of expert sexp[r] (tables of
+// L*d/2 entries, back to back) or, with sexp == nullptr, the single table
+// `coef`.  Must be called by all threads of the block (has __syncthreads).
 __device__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int *sexp, const float2 *coef,
                           bool transpose)
 {
+    const size_t estride = (size_t)L * (d >> 1);
     const int npass = (L + 4) / 5;
     for (int q = 0; q < npass; ++q) {
         const int pi = transpose ? (npass - 1 - q) : q;
         const int s0 = pi * L / npass;
         const int s1 = (pi + 1) * L / npass;
         if (transpose)
-            bfly_pass_g<true>(s1 - s0, tile, ld, rows, d, L, s0, sexp, coef, blockDim.x);
+            bfly_pass_g<true>(s1 - s0, tile, ld, rows, d, s0, sexp, coef, estride, blockDim.x);
         else
-            bfly_pass_g<false>(s1 - s0, tile, ld, rows, d, L, s0, sexp, coef, blockDim.x);
+            bfly_pass_g<false>(s1 - s0, tile, ld, rows, d, s0, sexp, coef, estride, blockDim.x);
         __syncthreads();
     }
 }

@@ -1,0 +1,263 @@
+// contract.cuh -- the ternary contraction of all routed rows against the one
+// shared W_base on the 5th-generation tensor cores, with the expert output
+// rotation fused into the epilogue.
+//
+// Z = X' W_base^T for every routed row at once (M = rows in bucket order,
+// N = K = d): W_base is shared by all experts, so the experts differ only in
+// the rotations around this single GEMM (ButterflyMoE summaries, section 2 /
+// 2.1: experts are never materialised; the ternary product "needs only
+// additions", section 3 -- on a tensor core the {-1, 0, +1} operand is exact
+// in fp16).
+//
+// Work unit = (128-row tile, BN-column slice of the output), BN = min(d, 256).
+// Persistent CTAs walk the units.  Warp roles:
+//   warp 0   one thread streams the A and W operand blocks with bulk copies
+//            through a kStages-deep shared-memory ring;
+//   warp 1   one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of
+//            two TMEM accumulators (double buffered: 2 x BN columns);
+//   warps 2-5  the epilogue: TMEM lane = tile row = thread, so each thread
+//            applies the output-butterfly stages that stay inside the slice
+//            (stages 0 .. log2 BN - 1) to its own row, with the row's expert
+//            table, and stores the fp32 result to the row's token-order slot.
+//            Stages 0-4 act inside 32-column blocks (one 32-column TMEM load,
+//            rotate, store back); stages 5.. act on columns 32 apart (4-column
+//            TMEM loads).  The remaining stages, which mix slices, are
+//            applied by the combine kernel.
+#pragma once
+
+#include "common.cuh"
+#include "layer.cuh"
+
+namespace bfmoe {
+
+constexpr int kContractThreads = 192;
+constexpr int kStages = 4;
+
+struct ContractParams {
+    const __half *a_blocks;   // [Rp/128][d/64] blocks of 128 x 64
+    const __half *w_blocks;   // [d/BN][d/64] blocks of BN x 64
+    float *slot;              // [R][d] fp32, token order (row i = t*k + j)
+    const int32_t *perm;      // bucket position -> i
+    const int32_t *topk_idx;  // i -> expert
+    const float2 *coef_p;     // [N][L][d/2] {cos, sin} of phi
+    int d, L, N, R, Rp;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void rot(float &a, float &b, float2 cs)
+{
+    const float x = a, y = b;
+    a = fmaf(cs.x, x, -(cs.y * y));
+    b = fmaf(cs.y, x, cs.x * y);
+}
+
+// Output-butterfly stages 0 .. log2(BN)-1 of one row held in TMEM columns
+// [tcol, tcol + BN) of this warp's lanes, then store to `out` (if non-null).
+template <int BN>
+__device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__restrict__ cf, int half,
+                                             float *__restrict__ out)
+{
+    constexpr int SIN = BN == 256 ? 8 : (BN == 128 ? 7 : 6);  // log2 BN
+    constexpr int G2 = SIN - 5;                              // stages at stride >= 32
+    constexpr int M2 = 1 << G2;
+    // pass 1: stages 0..4 inside each 32-column block
+#pragma unroll 1
+    for (int blk = 0; blk < BN / 32; ++blk) {
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)(blk * 32), v);
+#pragma unroll
+        for (int s = 0; s < 5; ++s) {
+            const float2 *cs = cf + (size_t)s * half;
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                if (m & (1 << s)) continue;
+                const int jj = blk * 32 + m;
+                const int pl = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
+                rot(v[m], v[m + (1 << s)], __ldg(cs + pl));
+            }
+        }
+        tmem_st32(tbase + (uint32_t)(blk * 32), v);
+    }
+    tmem_st_wait();
+    // pass 2: stages 5..SIN-1 on columns c + 32 m
+#pragma unroll 1
+    for (int c0 = 0; c0 < 32; c0 += 4) {
+        float v[4][M2];
+#pragma unroll
+        for (int m = 0; m < M2; ++m)
+            tmem_ld4_nowait(tbase + (uint32_t)(c0 + 32 * m), v[0][m], v[1][m], v[2][m], v[3][m]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int ls = 0; ls < G2; ++ls) {
+            const int s = 5 + ls;
+            const float2 *cs = cf + (size_t)s * half;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                for (int m = 0; m < M2; ++m) {
+                    if (m & (1 << ls)) continue;
+                    const int jj = c0 + q + 32 * m;
+                    const int pl = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
+                    rot(v[q][m], v[q][m + (1 << ls)], __ldg(cs + pl));
+                }
+            }
+        }
+        if (out) {
+#pragma unroll
+            for (int m = 0; m < M2; ++m)
+                *reinterpret_cast<float4 *>(out + c0 + 32 * m) = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+        }
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int d = p.d;
+    const int KC = d / kBK;
+    const int NH = d / BN;
+    const int MT = p.Rp / kBM;
+    const int nunits = MT * NH;
+    const int half = d >> 1;
+    constexpr uint32_t a_bytes = kBM * kBK * 2, b_bytes = (uint32_t)BN * kBK * 2;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + (size_t)kStages * a_bytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + (size_t)kStages * b_bytes);
+    uint64_t *full = bars, *empty = bars + kStages;
+    uint64_t *tfull = bars + 2 * kStages, *tempty = tfull + 2, *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the A blocks come from the input-butterfly kernel
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int it = 0;
+            for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x) {
+                const int mt = u / NH, nh = u % NH;
+                const __half *a_src = p.a_blocks + (size_t)mt * KC * (kBM * kBK);
+                const __half *b_src = p.w_blocks + (size_t)nh * KC * ((size_t)BN * kBK);
+                for (int kc = 0; kc < KC; ++kc, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u)) {
+                        set_status(p.status, BFMOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+                    bulk_g2s(sA + (size_t)s * a_bytes, a_src + (size_t)kc * (kBM * kBK), a_bytes, &full[s]);
+                    bulk_g2s(sB + (size_t)s * b_bytes, b_src + (size_t)kc * ((size_t)BN * kBK), b_bytes, &full[s]);
+                }
+            }
+            // every copy issued must have landed before the CTA exits
+            for (int q = it - kStages > 0 ? it - kStages : 0; q < it; ++q)
+                if (!mbar_wait(&full[q % kStages], (uint32_t)(q / kStages) & 1u)) set_status(p.status, BFMOE_ERR_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16_f32(kBM, BN);
+            int it = 0, li = 0;
+            for (int u = blockIdx.x; u < nunits && !*abort_flag; u += gridDim.x, ++li) {
+                const int b = li & 1;
+                if (!mbar_wait(&tempty[b], ((uint32_t)(li >> 1) & 1u) ^ 1u)) {
+                    set_status(p.status, BFMOE_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dcol = tmem + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kc = 0; kc < KC; ++kc, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u)) {
+                        set_status(p.status, BFMOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_addr(sA + (size_t)s * a_bytes), b0 = smem_addr(sB + (size_t)s * b_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t ad = sdesc_noswizzle(a0 + kk * 256, 128, 1024);
+                        const uint64_t bd = sdesc_noswizzle(b0 + kk * 256, 128, 1024);
+                        mma_f16(dcol, ad, bd, idesc, (kc | kk) != 0);
+                    }
+                    mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&tfull[b]);
+            }
+            // drain: wait until every MMA issued above has completed
+            mma_commit(drain);
+            if (!mbar_wait(drain, 0)) set_status(p.status, BFMOE_ERR_TIMEOUT);
+        }
+    } else {
+        // epilogue warps 2..5 own TMEM lanes 32*(warp % 4) .. +31
+        const int lane_base = (warp & 3) * 32;
+        int li = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++li) {
+            const int b = li & 1;
+            bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                if (lane == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
+                break;
+            }
+            tc_fence_after();
+            const int mt = u / NH, nh = u % NH;
+            const int r = mt * kBM + lane_base + lane;
+            int i = -1, e = 0;
+            if (r < p.R) {
+                i = p.perm[r];
+                if (i < 0 || i >= p.R) i = -1;
+                else e = min(max(p.topk_idx[i], 0), p.N - 1);
+            }
+            const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)nh * (BN / 2);
+            float *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
+            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, half, out);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+}
+
+__host__ inline size_t contract_smem_bytes(int d)
+{
+    const int BN = gemm_bn(d);
+    return 1024 + (size_t)kStages * (kBM * kBK * 2 + (size_t)BN * kBK * 2) + (2 * kStages + 5) * 8 + 16;
+}
+
+}  // namespace bfmoe

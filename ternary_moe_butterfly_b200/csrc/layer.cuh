@@ -1,18 +1,26 @@
-// layer.cuh -- the expert-layer kernels other than routing:
-//   k_pack_base      int8 ternary W_base -> 2-bit packed base (+ header)
-//   k_decode_base    packed base -> fp16 B-operand blocks for the GEMM
-//   k_coef           angles -> {cos, sin} tables
-//   k_expert_in      gather routed rows by bucket, input rotation B(theta)^T,
-//                    fp16 A-operand blocks
-//   k_contract       ONE tcgen05 GEMM of all routed rows against W_base
-//   k_expert_out     output rotation B(phi), alpha * gate, combine per token
-//   k_bfly_apply     standalone row butterfly (B or B^T)
+// layer.cuh -- the expert-layer kernels around the contraction:
+//   k_pack_base    int8 ternary W_base -> 2-bit packed words
+//   k_expert_in    gather each single-expert tile of bucketed rows, input
+//                  rotation B(theta_e)^T, fp16 operand blocks for the GEMM
+//   k_combine      output stages the GEMM epilogue could not reach (those
+//                  that mix columns 256 or more apart), alpha * gate, and
+//                  the per-token sum over the k routed rows
+//   k_bfly_apply   standalone row butterfly (B or B^T)
 //
 // The method: expert i is W_i = alpha B(phi_i) W_base B(theta_i)^T with a
 // single shared ternary W_base and per-expert butterflies; W_i is never
 // formed -- input rotation, ternary product, output rotation in sequence
 // (ButterflyMoE summaries, section 2 / 2.1; ButterflyViT summary, section 2).
-//
+#pragma once
+
+#include "butterfly.cuh"
+#include "common.cuh"
+#include "route.cuh"
+
+namespace bfmoe {
+
+constexpr int kBM = 128;  // GEMM rows per tile (tcgen05 M)
+
 // GEMM operand layout ("blocks"): a matrix with rows m and contraction index
 // k is stored as blocks of 64 k-columns; block (mt, kc) holds rows
 // [mt*BR, mt*BR + BR) x k in [64 kc, 64 kc + 64) as 8x8 core matrices of
@@ -21,20 +29,6 @@
 // contiguous bulk copy into shared memory, already in the tensor core's
 // canonical K-major no-swizzle layout (core matrices 128 B apart along K,
 // 1024 B apart along M).
-#pragma once
-
-#include "butterfly.cuh"
-#include "common.cuh"
-
-namespace bfmoe {
-
-constexpr int kBM = 128;          // GEMM rows per tile (tcgen05 M)
-constexpr int kBK = 64;           // contraction columns per pipeline stage
-constexpr int kGemmStages = 4;
-constexpr uint32_t kPackMagic = 0x32574642u;  // "BFW2"
-
-__host__ __device__ constexpr int gemm_bn(int d) { return d < 256 ? d : 256; }
-
 __device__ __forceinline__ size_t block_elem_offset(int m, int k, int BR, int KC)
 {
     const int mt = m / BR, mi = m % BR, kc = k / kBK, ki = k % kBK;
@@ -66,56 +60,17 @@ __global__ void k_pack_base(const int8_t *__restrict__ w, int d, uint32_t *__res
     if (!ok) atomicOr(bad, 1u);
 }
 
-// Packed base -> fp16 B blocks (rows = output index n, contraction = k).
-// One thread per 16-byte chunk (8 consecutive k of one row).
-__global__ void k_decode_base(const uint32_t *__restrict__ packed, int d, __half *__restrict__ wb,
-                              uint32_t *status)
-{
-    const int BN = gemm_bn(d);
-    const int KC = d / kBK;
-    const size_t nchunks = (size_t)d * d / 8;
-    const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (q == 0 && (packed[0] != kPackMagic || packed[1] != (uint32_t)d)) set_status(status, BFMOE_ERR_INVALID_ARG);
-    if (q >= nchunks) return;
-    // q enumerates chunks in memory order of the block layout
-    const size_t blk = q / ((size_t)BN * 8);
-    const int within = (int)(q % ((size_t)BN * 8));
-    const int core = within >> 3, rr = within & 7;
-    const int nt = (int)(blk / KC), kc = (int)(blk % KC);
-    const int n = nt * BN + ((core >> 3) << 3) + rr;
-    const int k0 = kc * kBK + ((core & 7) << 3);
-    const uint32_t word = packed[4 + (size_t)n * (d / 16) + (k0 >> 4)];
-    const uint32_t bits = word >> (2 * (k0 & 15));
-    uint32_t h[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t c0 = (bits >> (4 * i)) & 3u, c1 = (bits >> (4 * i + 2)) & 3u;
-        // 01 -> +1 (0x3C00), 11 -> -1 (0xBC00), 00 / 10 -> 0
-        const uint32_t lo = c0 == 1u ? 0x3C00u : (c0 == 3u ? 0xBC00u : 0u);
-        const uint32_t hi = c1 == 1u ? 0x3C00u : (c1 == 3u ? 0xBC00u : 0u);
-        h[i] = lo | (hi << 16);
-    }
-    reinterpret_cast<uint4 *>(wb)[q] = make_uint4(h[0], h[1], h[2], h[3]);
-}
-
-// --------------------------------------------------------------- angles --
-
-__global__ void k_coef(const float *__restrict__ a0, const float *__restrict__ a1, int count,
-                       float2 *__restrict__ c0, float2 *__restrict__ c1)
+__global__ void k_coef(const float *__restrict__ a, int count, float2 *__restrict__ c)
 {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < count) {
-        float s, c;
-        sincosf(a0[i], &s, &c);
-        c0[i] = make_float2(c, s);
-    } else if (a1 && i < 2 * count) {
-        float s, c;
-        sincosf(a1[i - count], &s, &c);
-        c1[i - count] = make_float2(c, s);
+        float s, co;
+        sincosf(a[i], &s, &co);
+        c[i] = make_float2(co, s);
     }
 }
 
-// ------------------------------------------------------- tile row loads --
+// ------------------------------------------------------- tile row I/O --
 
 // Load one row of d values of type T into a tile row (fp32), cooperatively
 // by one warp with 16-byte loads.
@@ -147,188 +102,6 @@ __device__ __forceinline__ void warp_load_row<__nv_bfloat16>(const __nv_bfloat16
     }
 }
 
-// ---------------------------------------------------------- input side --
-
-// Rows r in [blockIdx.x*RT, +RT) of the bucket-sorted row list: gather x of
-// the row's token, rotate by B(theta_e)^T, write fp16 A blocks.  Rows >= R
-// (tile padding) are written as zeros.
-template <typename T>
-__global__ void __launch_bounds__(256) k_expert_in(const T *__restrict__ x, int d, int L, int k, int R,
-                                                   const int32_t *__restrict__ perm,
-                                                   const int32_t *__restrict__ topk_idx,
-                                                   const float2 *__restrict__ coef_theta, __half *__restrict__ a_blocks,
-                                                   uint32_t *status)
-{
-    extern __shared__ float tile[];
-    const int RT = tile_rows_for(d);
-    const int ld = d + 1;
-    int *sexp = reinterpret_cast<int *>(tile + (size_t)RT * ld);
-    int *stok = sexp + RT;
-    const int r0 = blockIdx.x * RT;
-    if (threadIdx.x < RT) {
-        const int r = r0 + threadIdx.x;
-        int e = 0, t = -1;
-        if (r < R) {
-            const int i = perm[r];
-            t = i / k;
-            e = topk_idx[i];
-        }
-        sexp[threadIdx.x] = e;
-        stok[threadIdx.x] = t;
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int q = warp; q < RT; q += nw) {
-        const int t = stok[q];
-        float *dst = tile + (size_t)q * ld;
-        if (t >= 0)
-            warp_load_row<T>(x + (size_t)t * d, dst, d, lane);
-        else
-            for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
-    }
-    __syncthreads();
-    bfly_tile(tile, ld, RT, d, L, sexp, coef_theta, /*transpose=*/true);
-    // fp16 A blocks: one thread per (row, 8-column chunk), rows fastest.
-    const int KC = d / kBK;
-    const int nch = RT * (d / 8);
-    bool overflow = false;
-    for (int q = threadIdx.x; q < nch; q += blockDim.x) {
-        const int rq = q % RT, c8 = q / RT;
-        const float *src = tile + (size_t)rq * ld + c8 * 8;
-        float f[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            f[i] = src[i];
-            overflow |= !(fabsf(f[i]) <= 65504.0f);
-        }
-        const size_t off = block_elem_offset(r0 + rq, c8 * 8, kBM, KC);
-        *reinterpret_cast<uint4 *>(a_blocks + off) = pack_f16x8(f);
-    }
-    if (overflow) set_status(status, BFMOE_ERR_NONFINITE);
-}
-
-// ----------------------------------------------------------- contraction --
-
-// Z[m][n] = sum_k A[m][k] * W[n][k] for one 128 x BN tile, fp16 operands,
-// fp32 accumulation in tensor memory.  Thread 0 streams the A and W blocks
-// with bulk copies through a kGemmStages-deep ring; thread 32 issues the
-// tcgen05.mma instructions; all four warps drain the accumulator (warp w
-// owns TMEM lanes 32w..32w+31 = tile rows 32w..32w+31) to fp32 Z.
-__global__ void __launch_bounds__(128, 1) k_contract(const __half *__restrict__ a_blocks,
-                                                     const __half *__restrict__ w_blocks, float *__restrict__ z,
-                                                     int d, uint32_t *status)
-{
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const int BN = gemm_bn(d);
-    const int KC = d / kBK;
-    const int S = KC < kGemmStages ? KC : kGemmStages;
-    const uint32_t a_bytes = kBM * kBK * 2, b_bytes = (uint32_t)BN * kBK * 2;
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;
-    uint8_t *sB = smem + (size_t)S * a_bytes;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + (size_t)S * b_bytes);
-    uint64_t *full = bars, *empty = bars + kGemmStages, *done = bars + 2 * kGemmStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGemmStages + 1);
-    volatile uint32_t *abort_flag = tmem_slot + 1;
-
-    const int mt = blockIdx.x, nt = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kGemmStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(done, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) tmem_alloc(tmem_slot, (uint32_t)BN);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (threadIdx.x == 0) {
-        // producer
-        const __half *a_src = a_blocks + (size_t)mt * KC * (kBM * kBK);
-        const __half *b_src = w_blocks + (size_t)nt * KC * ((size_t)BN * kBK);
-        int issued = 0;
-        for (int kc = 0; kc < KC; ++kc) {
-            const int s = kc % S;
-            const uint32_t ph = (uint32_t)(kc / S) & 1u;
-            if (!mbar_wait(&empty[s], ph ^ 1u)) {
-                set_status(status, BFMOE_ERR_TIMEOUT);
-                *abort_flag = 1;
-                break;
-            }
-            if (*abort_flag) break;
-            mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
-            bulk_g2s(sA + (size_t)s * a_bytes, a_src + (size_t)kc * (kBM * kBK), a_bytes, &full[s]);
-            bulk_g2s(sB + (size_t)s * b_bytes, b_src + (size_t)kc * ((size_t)BN * kBK), b_bytes, &full[s]);
-            issued = kc + 1;
-        }
-        // before leaving, every copy issued must have landed
-        for (int kc = issued - S > 0 ? issued - S : 0; kc < issued; ++kc)
-            if (!mbar_wait(&full[kc % S], (uint32_t)(kc / S) & 1u)) set_status(status, BFMOE_ERR_TIMEOUT);
-    } else if (threadIdx.x == 32) {
-        // MMA issuer
-        const uint32_t idesc = idesc_f16_f32(kBM, BN);
-        for (int kc = 0; kc < KC; ++kc) {
-            const int s = kc % S;
-            if (!mbar_wait(&full[s], (uint32_t)(kc / S) & 1u)) {
-                set_status(status, BFMOE_ERR_TIMEOUT);
-                *abort_flag = 1;
-                break;
-            }
-            if (*abort_flag) break;
-            tc_fence_after();
-            const uint32_t a0 = smem_addr(sA + (size_t)s * a_bytes), b0 = smem_addr(sB + (size_t)s * b_bytes);
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-                const uint64_t ad = sdesc_noswizzle(a0 + kk * 256, 128, 1024);
-                const uint64_t bd = sdesc_noswizzle(b0 + kk * 256, 128, 1024);
-                mma_f16(tmem, ad, bd, idesc, (kc | kk) != 0);
-            }
-            mma_commit(&empty[s]);
-        }
-        mma_commit(done);  // arrives once every MMA issued above has completed
-    }
-    __syncwarp();
-    // epilogue: all 128 threads; every branch below is warp-uniform so the
-    // .sync.aligned TMEM loads see converged warps
-    bool ok = mbar_wait(done, 0);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok && lane == 0) set_status(status, BFMOE_ERR_TIMEOUT);
-    tc_fence_after();
-    const bool aborted = __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
-    if (ok && !aborted) {
-        const int row = mt * kBM + warp * 32 + lane;
-        float *zrow = z + (size_t)row * d + (size_t)nt * BN;
-        for (int c = 0; c < BN; c += 32) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(zrow + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, (uint32_t)BN);
-}
-
-__host__ inline size_t contract_smem_bytes(int d)
-{
-    const int BN = gemm_bn(d);
-    const int KC = d / kBK;
-    const int S = KC < kGemmStages ? KC : kGemmStages;
-    return 1024 + (size_t)S * (kBM * kBK * 2 + (size_t)BN * kBK * 2) + (2 * kGemmStages + 1) * 8 + 16;
-}
-
-// ---------------------------------------------------------- output side --
-
-// Tokens [blockIdx.x*TT, +TT): for each routed row (t, j) read Z at its
-// bucket position, rotate by B(phi_e), then y_t = alpha sum_j g_j u_j.
 template <typename T>
 __device__ __forceinline__ void store8(T *dst, const float *f);
 template <>
@@ -343,68 +116,197 @@ __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 *dst, const 
     *reinterpret_cast<uint4 *>(dst) = pack_bf16x8(f);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) k_expert_out(const float *__restrict__ z, int d, int L, int T_, int k,
-                                                    const int32_t *__restrict__ row_pos,
-                                                    const int32_t *__restrict__ topk_idx,
-                                                    const float *__restrict__ gates,
-                                                    const float2 *__restrict__ coef_phi,
-                                                    const uint32_t *__restrict__ packed, T *__restrict__ y)
+__device__ __forceinline__ void store1(float *dst, float v) { *dst = v; }
+__device__ __forceinline__ void store1(__nv_bfloat16 *dst, float v) { *dst = __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------- input side --
+
+struct ExpertInParams {
+    const void *x;
+    int d, L, k, N, R;
+    const int32_t *perm;
+    const int4 *tiles;       // single-expert row tiles {expert, row0, nrows, -}
+    const int32_t *n_tiles;
+    int max_tiles;           // capacity of `tiles`
+    const float2 *coef_t;    // [N][L][d/2] {cos, sin} of theta
+    __half *a_blocks;        // fp16 operand blocks, rows in bucket order
+    uint32_t *status;
+};
+
+// Persistent over the tile list: gather the rows of one expert's tile, rotate
+// by B(theta_e)^T (the expert's cos/sin table is staged in shared memory when
+// it fits, so every coefficient load is a broadcast), write fp16 A blocks.
+template <typename T, bool SMEM_COEF>
+__global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
 {
-    extern __shared__ float tile[];
-    const int RT0 = tile_rows_for(d);
-    const int TT = RT0 / k > 0 ? RT0 / k : 1;
-    const int RT = TT * k;
+    extern __shared__ __align__(16) float smem_f[];
+    const int d = p.d, L = p.L;
+    const int RT = tile_rows_for(d);
     const int ld = d + 1;
-    int *sexp = reinterpret_cast<int *>(tile + (size_t)RT * ld);
-    int *spos = sexp + RT;
-    float *sg = reinterpret_cast<float *>(spos + RT);
-    const int t0 = blockIdx.x * TT;
-    if (threadIdx.x < RT) {
-        const int t = t0 + threadIdx.x / k;
-        int e = 0, pos = -1;
-        float g = 0.0f;
-        if (t < T_) {
-            const int i = t * k + threadIdx.x % k;
-            pos = row_pos[i];
-            e = topk_idx[i];
-            g = gates[i];
-        }
-        sexp[threadIdx.x] = e;
-        spos[threadIdx.x] = pos;
-        sg[threadIdx.x] = g;
-    }
-    __syncthreads();
+    const size_t tab = (size_t)L * (d >> 1);
+    float2 *sc = reinterpret_cast<float2 *>(smem_f);  // [tab] when SMEM_COEF
+    float *tile = smem_f + (SMEM_COEF ? 2 * tab : 0);
+    int *stok = reinterpret_cast<int *>(tile + (size_t)RT * ld);
+    pdl_wait();
+    pdl_trigger();
+    // a routing that gave up (timeout) leaves the list unspecified: clamp it
+    const int ntiles = min(max(*p.n_tiles, 0), p.max_tiles);
+    const T *x = reinterpret_cast<const T *>(p.x);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int q = warp; q < RT; q += nw) {
-        const int pos = spos[q];
-        float *dst = tile + (size_t)q * ld;
-        if (pos >= 0)
-            warp_load_row<float>(z + (size_t)pos * d, dst, d, lane);
-        else
-            for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
+    const int KC = d / kBK;
+    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+        const int4 tl = p.tiles[ti];
+        const int e = min(max(tl.x, 0), p.N - 1);
+        const int r0 = tl.y;
+        int nr = min(max(tl.z, 0), RT);
+        if (r0 < 0 || r0 > p.R - nr) nr = 0;
+        if (nr == 0) continue;  // uniform across the block
+        const float2 *gtab = p.coef_t + (size_t)e * tab;
+        if (SMEM_COEF) {
+            const float4 *src = reinterpret_cast<const float4 *>(gtab);
+            float4 *dst = reinterpret_cast<float4 *>(sc);
+            for (size_t q = threadIdx.x; q < tab / 2; q += blockDim.x) dst[q] = __ldg(src + q);
+        }
+        if ((int)threadIdx.x < RT) {
+            int t = -1;
+            const int r = r0 + (int)threadIdx.x;
+            if ((int)threadIdx.x < nr && r >= 0 && r < p.R) {
+                const int i = p.perm[r];
+                if (i >= 0 && i < p.R) t = i / p.k;
+            }
+            stok[threadIdx.x] = t;
+        }
+        __syncthreads();
+        for (int q = warp; q < nr; q += nw) {
+            const int t = stok[q];
+            float *dst = tile + (size_t)q * ld;
+            if (t >= 0)
+                warp_load_row<T>(x + (size_t)t * d, dst, d, lane);
+            else
+                for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
+        }
+        __syncthreads();
+        bfly_tile(tile, ld, nr, d, L, nullptr, SMEM_COEF ? sc : gtab, /*transpose=*/true);
+        bool overflow = false;
+        const int nch = nr * (d / 8);
+        for (int q = threadIdx.x; q < nch; q += blockDim.x) {
+            const int rq = q % nr, c8 = q / nr;
+            const float *src = tile + (size_t)rq * ld + c8 * 8;
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                f[i] = src[i];
+                overflow |= !(fabsf(f[i]) <= 65504.0f);
+            }
+            const size_t off = block_elem_offset(r0 + rq, c8 * 8, kBM, KC);
+            *reinterpret_cast<uint4 *>(p.a_blocks + off) = pack_f16x8(f);
+        }
+        if (overflow) set_status(p.status, BFMOE_ERR_NONFINITE);
+        __syncthreads();
     }
-    __syncthreads();
-    bfly_tile(tile, ld, RT, d, L, sexp, coef_phi, /*transpose=*/false);
-    const float alpha = __uint_as_float(packed[2]);
-    const int nch = TT * (d / 8);
-    for (int q = threadIdx.x; q < nch; q += blockDim.x) {
-        const int tt = q / (d / 8), c8 = q % (d / 8);
-        const int t = t0 + tt;
-        if (t >= T_) continue;
-        float f[8];
+}
+
+__host__ inline size_t expert_in_smem_bytes(int d, int L, bool smem_coef)
+{
+    const int RT = tile_rows_for(d);
+    return (smem_coef ? (size_t)L * (d / 2) * 8 : 0) + (size_t)RT * (d + 1) * 4 + (size_t)RT * 4;
+}
+
+__host__ inline bool expert_in_smem_coef(int d, int L) { return (size_t)L * (d / 2) * 8 <= 40 * 1024; }
+
+// ------------------------------------------------------------ combine --
+
+struct CombineParams {
+    const float *slot;        // [T*k][d] fp32, rows in token order (i = t*k + j)
+    int T, d, L, k, N;
+    int s_lo;                 // first output stage left to apply (log2 of the GEMM's N tile)
+    const int32_t *topk_idx;
+    const float *gates;
+    const float2 *coef_p;     // [N][L][d/2]
+    const uint32_t *packed;   // alpha in word 2
+    void *y;
+};
+
+// HS = L - s_lo > 0 high stages: one token per block, 256 threads; thread c
+// owns columns c + 256 m (m < 2^HS), which the stages s_lo..L-1 mix.
+template <typename T, int HS>
+__global__ void __launch_bounds__(256) k_combine_high(CombineParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    constexpr int G = 1 << HS;
+    const int t = blockIdx.x;
+    if (t >= p.T) return;
+    const int c = threadIdx.x;
+    const int d = p.d, half = d >> 1;
+    float acc[G];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const float *src = tile + (size_t)(tt * k + j) * ld + c8 * 8;
-            const float g = sg[tt * k + j];
+    for (int m = 0; m < G; ++m) acc[m] = 0.0f;
+    for (int j = 0; j < p.k; ++j) {
+        const int i = t * p.k + j;
+        const int e = min(max(p.topk_idx[i], 0), p.N - 1);
+        const float g = p.gates[i];
+        const float *row = p.slot + (size_t)i * d;
+        float v[G];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = fmaf(g, src[i], f[i]);
+        for (int m = 0; m < G; ++m) v[m] = row[c + 256 * m];
+        const float2 *cf = p.coef_p + (size_t)e * p.L * half;
+#pragma unroll
+        for (int ls = 0; ls < HS; ++ls) {
+            const int s = p.s_lo + ls;
+            const float2 *cs = cf + (size_t)s * half;
+#pragma unroll
+            for (int m = 0; m < G; ++m) {
+                if (m & (1 << ls)) continue;
+                const int jj = c + 256 * m;
+                const int pp = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
+                const float2 cs2 = __ldg(cs + pp);
+                const float a = v[m], b = v[m + (1 << ls)];
+                v[m] = fmaf(cs2.x, a, -(cs2.y * b));
+                v[m + (1 << ls)] = fmaf(cs2.y, a, cs2.x * b);
+            }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] *= alpha;
-        store8<T>(y + (size_t)t * d + c8 * 8, f);
+        for (int m = 0; m < G; ++m) acc[m] = fmaf(g, v[m], acc[m]);
     }
+    const float alpha = __uint_as_float(__ldg(p.packed + 2));
+    T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d;
+#pragma unroll
+    for (int m = 0; m < G; ++m) store1(y + c + 256 * m, alpha * acc[m]);
+}
+
+// No stage left (d <= 256): 8 columns per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) k_combine_sum(CombineParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int d = p.d;
+    const int per_tok = d / 8;
+    const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int t = (int)(q / per_tok), c8 = (int)(q % per_tok);
+    if (t >= p.T) return;
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = 0.0f;
+    for (int j = 0; j < p.k; ++j) {
+        const int i = t * p.k + j;
+        const float g = p.gates[i];
+        const float4 *src = reinterpret_cast<const float4 *>(p.slot + (size_t)i * d + c8 * 8);
+        const float4 a = src[0], b = src[1];
+        f[0] = fmaf(g, a.x, f[0]);
+        f[1] = fmaf(g, a.y, f[1]);
+        f[2] = fmaf(g, a.z, f[2]);
+        f[3] = fmaf(g, a.w, f[3]);
+        f[4] = fmaf(g, b.x, f[4]);
+        f[5] = fmaf(g, b.y, f[5]);
+        f[6] = fmaf(g, b.z, f[6]);
+        f[7] = fmaf(g, b.w, f[7]);
+    }
+    const float alpha = __uint_as_float(__ldg(p.packed + 2));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] *= alpha;
+    store8<T>(reinterpret_cast<T *>(p.y) + (size_t)t * d + c8 * 8, f);
 }
 
 // ------------------------------------------------------ standalone rows --

@@ -1,5 +1,5 @@
 // route.cuh -- top-k gate over given router logits and deterministic
-// bucketing of the routed rows by expert.
+// bucketing of the routed rows by expert, in ONE cooperative kernel.
 //
 // A standard top-k gate selects each token's active experts (ButterflyMoE
 // summary, Dutch page, section 2 "Three phases", gated routing).  Order:
@@ -7,10 +7,19 @@
 // the k selected logits.  Bucketing is a stable counting sort of the rows
 // i = t*k + j by expert, so each bucket lists its rows in token order.
 //
-// Three launches: (1) one warp per token selects the top-k and counts the
-// block's rows per expert; (2) one block turns the per-block counts into
-// bucket offsets and per-block bases; (3) per block, one warp ranks the
-// block's rows inside their buckets (warp match + popcount) and scatters.
+// Phases, separated by two bounded grid barriers (all blocks are
+// co-resident: the kernel is launched cooperatively):
+//   A  one warp per token selects the top-k; each 64-token chunk counts its
+//      rows per expert (hist[chunk][e]).  While the routing runs, the same
+//      blocks also turn the butterfly angles into {cos, sin} tables and
+//      decode the packed ternary base into the tensor-core operand layout
+//      (forward only).
+//   B  one warp per expert scans hist[.][e] over the chunks (exclusive
+//      prefix per chunk, total per expert).
+//   C  every block scans the expert totals into bucket offsets, then ranks
+//      the rows of its chunks inside their buckets (warp match + popcount)
+//      and scatters perm / row_pos; the blocks also write the list of
+//      single-expert row tiles that the input-butterfly kernel walks.
 #pragma once
 
 #include "common.cuh"
@@ -18,8 +27,38 @@
 namespace bfmoe {
 
 constexpr int kRouteThreads = 256;
-constexpr int kRouteTokensPerBlock = 64;  // 8 warps x 8 tokens
+constexpr int kRouteChunk = 64;  // tokens per chunk: 8 warps x 8 tokens
 constexpr int kMaxK = 8;
+constexpr uint32_t kPackMagic = 0x32574642u;  // "BFW2"
+
+__host__ __device__ constexpr int gemm_bn(int d) { return d < 256 ? d : 256; }
+constexpr int kBK = 64;  // contraction columns per GEMM operand block
+
+struct RouteParams {
+    const float *logits;
+    int T, N, k;
+    int32_t *topk_idx;   // [T][k]
+    float *gates;        // [T][k]
+    int32_t *perm;       // [T*k]
+    int32_t *row_pos;    // [T*k] or null
+    int32_t *offsets;    // [N+1]
+    int32_t *hist;       // [nchunk][N] -> per-chunk bucket bases
+    int32_t *total;      // [N]
+    uint32_t *sync;      // grid barrier counter, zero at launch
+    uint32_t *status;
+    int skip_arrive_block;  // test hook: this block never reaches barrier 1 (-1: none)
+    // forward only: prep done while routing
+    const float *theta, *phi;
+    float2 *coef_t, *coef_p;
+    int ncoef;
+    const uint32_t *packed;
+    __half *wdec;
+    int d;
+    // forward only: single-expert row tiles for the input butterfly
+    int4 *in_tiles;
+    int32_t *n_in_tiles;
+    int tile_rows;
+};
 
 // (va, a) ranks before (vb, b)?  NaN has been mapped to -inf by the caller.
 __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b)
@@ -27,30 +66,56 @@ __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b)
     return va > vb || (va == vb && a < b);
 }
 
-__global__ void __launch_bounds__(kRouteThreads) k_topk(const float *__restrict__ logits, int T, int N, int k,
-                                                        int32_t *__restrict__ topk_idx,
-                                                        float *__restrict__ gates, int32_t *__restrict__ hist,
-                                                        uint32_t *status)
+// Bounded grid-wide barrier on a monotonically increasing counter.  Returns
+// false (block-uniformly) if the other blocks did not arrive in time.
+__device__ bool grid_barrier(uint32_t *ctr, uint32_t target, uint32_t *status, bool arrive)
 {
-    extern __shared__ int sh_hist[];  // [N]
+    __shared__ int ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ok = 1;
+        __threadfence();
+        if (arrive) atomicAdd(ctr, 1u);
+        const unsigned long long t0 = globaltimer_ns();
+        while (true) {
+            const uint32_t v = *reinterpret_cast<volatile uint32_t *>(ctr);
+            if (v >= target) break;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                set_status(status, BFMOE_ERR_TIMEOUT);
+                ok = 0;
+                break;
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return ok != 0;
+}
+
+// Top-k, gates and the chunk histogram for tokens [c*64, c*64+64).
+__device__ void topk_chunk(const RouteParams &p, int c, int *sh_hist, bool &saw_nan)
+{
+    const int N = p.N, k = p.k;
     for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
     __syncthreads();
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tok0 = blockIdx.x * kRouteTokensPerBlock + warp * (kRouteTokensPerBlock / 8);
-    bool saw_nan = false;
-    for (int q = 0; q < kRouteTokensPerBlock / 8; ++q) {
+    const int tok0 = c * kRouteChunk + warp * (kRouteChunk / 8);
+    for (int q = 0; q < kRouteChunk / 8; ++q) {
         const int t = tok0 + q;
-        if (t >= T) break;
-        const float *l = logits + (size_t)t * N;
+        if (t >= p.T) break;
+        const float *l = p.logits + (size_t)t * N;
         int sel[kMaxK];
         float val[kMaxK];
-        for (int j = 0; j < k; ++j) {
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j >= k) break;
             float bv = -INFINITY;
             int be = 0x7fffffff;
             for (int e = lane; e < N; e += 32) {
                 bool taken = false;
-                for (int jj = 0; jj < j; ++jj) taken |= (sel[jj] == e);
+#pragma unroll
+                for (int jj = 0; jj < kMaxK; ++jj)
+                    if (jj < j) taken |= (sel[jj] == e);
                 if (taken) continue;
                 float v = __ldg(l + e);
                 if (v != v) {
@@ -78,9 +143,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_topk(const float *__restrict_
             float g[kMaxK];
             const float m = val[0];
             if (m == INFINITY) {
-                int c = 0;
-                for (int j = 0; j < k; ++j) c += (val[j] == INFINITY);
-                for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)c : 0.0f;
+                int cnt = 0;
+                for (int j = 0; j < k; ++j) cnt += (val[j] == INFINITY);
+                for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)cnt : 0.0f;
             } else if (m == -INFINITY) {
                 for (int j = 0; j < k; ++j) g[j] = 1.0f / (float)k;
             } else {
@@ -93,93 +158,185 @@ __global__ void __launch_bounds__(kRouteThreads) k_topk(const float *__restrict_
                 for (int j = 0; j < k; ++j) g[j] *= rz;
             }
             for (int j = 0; j < k; ++j) {
-                topk_idx[(size_t)t * k + j] = sel[j];
-                gates[(size_t)t * k + j] = g[j];
+                p.topk_idx[(size_t)t * k + j] = sel[j];
+                p.gates[(size_t)t * k + j] = g[j];
                 atomicAdd(&sh_hist[sel[j]], 1);
             }
         }
     }
-    if (__any_sync(0xffffffffu, saw_nan) && lane == 0) set_status(status, BFMOE_ERR_NONFINITE);
     __syncthreads();
-    for (int e = threadIdx.x; e < N; e += blockDim.x) hist[(size_t)blockIdx.x * N + e] = sh_hist[e];
+    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)c * N + e] = sh_hist[e];
+    __syncthreads();
 }
 
-// One block: base[b][e] = offsets[e] + sum_{b' < b} hist[b'][e] (in place),
-// offsets[e] = sum_{e' < e} total[e'], offsets[N] = R.
-__global__ void __launch_bounds__(1024) k_bucket_scan(int32_t *__restrict__ hist_base, int nblk, int N,
-                                                      int32_t *__restrict__ offsets)
+// Packed base -> fp16 B blocks for the contraction (rows = output index n,
+// contraction = k; see the operand layout in contract.cuh).  One call per
+// 16-byte output chunk q (8 consecutive k of one row).
+__device__ __forceinline__ void decode_chunk(const uint32_t *__restrict__ packed, int d, __half *__restrict__ wb,
+                                             size_t q)
 {
-    extern __shared__ int sh[];  // total[N] then scratch[1024]
-    int *total = sh;
-    int *part = sh + N;
-    for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        int run = 0;
-        for (int b = 0; b < nblk; ++b) {
-            const int h = hist_base[(size_t)b * N + e];
-            hist_base[(size_t)b * N + e] = run;
-            run += h;
-        }
-        total[e] = run;
+    const int BN = gemm_bn(d);
+    const int KC = d / kBK;
+    const size_t blk = q / ((size_t)BN * 8);
+    const int within = (int)(q % ((size_t)BN * 8));
+    const int core = within >> 3, rr = within & 7;
+    const int nt = (int)(blk / KC), kc = (int)(blk % KC);
+    const int n = nt * BN + ((core >> 3) << 3) + rr;
+    const int k0 = kc * kBK + ((core & 7) << 3);
+    const uint32_t word = __ldg(packed + 4 + (size_t)n * (d / 16) + (k0 >> 4));
+    const uint32_t bits = word >> (2 * (k0 & 15));
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t c0 = (bits >> (4 * i)) & 3u, c1 = (bits >> (4 * i + 2)) & 3u;
+        // 01 -> +1 (fp16 0x3C00), 11 -> -1 (0xBC00), 00 / 10 -> 0
+        const uint32_t lo = c0 == 1u ? 0x3C00u : (c0 == 3u ? 0xBC00u : 0u);
+        const uint32_t hi = c1 == 1u ? 0x3C00u : (c1 == 3u ? 0xBC00u : 0u);
+        h[i] = lo | (hi << 16);
     }
-    __syncthreads();
-    // exclusive scan of total[0..N) with 1024 threads, ceil(N/1024) items each
-    const int per = (N + blockDim.x - 1) / blockDim.x;
-    const int lo = threadIdx.x * per, hi = min(N, lo + per);
+    reinterpret_cast<uint4 *>(wb)[q] = make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// Exclusive scan of src[0..n) into dst[0..n) by the whole block; returns the
+// sum.  `scratch` holds blockDim.x ints.  src and dst may alias.
+__device__ int block_exclusive_scan(const int *src, int *dst, int n, int *scratch)
+{
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
     int s = 0;
-    for (int e = lo; e < hi; ++e) s += total[e];
-    part[threadIdx.x] = s;
+    for (int e = lo; e < hi; ++e) s += src[e];
+    scratch[threadIdx.x] = s;
     __syncthreads();
     for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-        const int v = (threadIdx.x >= (unsigned)off) ? part[threadIdx.x - off] : 0;
+        const int v = (int)threadIdx.x >= off ? scratch[threadIdx.x - off] : 0;
         __syncthreads();
-        part[threadIdx.x] += v;
+        scratch[threadIdx.x] += v;
         __syncthreads();
     }
-    int run = part[threadIdx.x] - s;  // exclusive prefix of this thread's range
+    int run = scratch[threadIdx.x] - s;
+    const int totalsum = scratch[blockDim.x - 1];
+    __syncthreads();
     for (int e = lo; e < hi; ++e) {
-        const int t = total[e];
-        total[e] = run;
-        run += t;
+        const int v = src[e];
+        dst[e] = run;
+        run += v;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < N; e += blockDim.x) offsets[e] = total[e];
-    if (threadIdx.x == blockDim.x - 1) offsets[N] = part[blockDim.x - 1];
-    for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        const int o = total[e];
-        for (int b = 0; b < nblk; ++b) hist_base[(size_t)b * N + e] += o;
-    }
+    return totalsum;
 }
 
-// Per block (same token partition as k_topk): rank the block's rows inside
-// their buckets in row order and scatter perm / row_pos.
-__global__ void __launch_bounds__(kRouteThreads) k_bucket_scatter(const int32_t *__restrict__ topk_idx,
-                                                                  const int32_t *__restrict__ base, int T, int N,
-                                                                  int k, int32_t *__restrict__ perm,
-                                                                  int32_t *__restrict__ row_pos)
+__global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
 {
-    extern __shared__ int cnt[];  // [N]
-    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = base[(size_t)blockIdx.x * N + e];
-    __syncthreads();
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
-    const int t0 = blockIdx.x * kRouteTokensPerBlock;
-    const int t1 = min(T, t0 + kRouteTokensPerBlock);
-    const int i0 = t0 * k, i1 = t1 * k;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int c0 = i0; c0 < i1; c0 += 32) {
-        const int i = c0 + lane;
-        const bool valid = i < i1;
-        const int e = valid ? topk_idx[i] : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int pos = valid ? cnt[e] + __popc(peers & lt) : 0;
-        __syncwarp();
-        if (valid && (__ffs(peers) - 1) == lane) cnt[e] += __popc(peers);
-        __syncwarp();
-        if (valid) {
-            perm[pos] = i;
-            if (row_pos) row_pos[i] = pos;
+    extern __shared__ int sh[];  // phase A: hist[N]; phase C: off[N+1], tstart[N+1], cnt[N], scratch[256]
+    const int N = p.N, k = p.k;
+    const int nchunk = (p.T + kRouteChunk - 1) / kRouteChunk;
+    const int R = p.T * k;
+
+    // ---- phase A: top-k and chunk histograms, plus the prep work
+    bool saw_nan = false;
+    for (int c = blockIdx.x; c < nchunk; c += gridDim.x) topk_chunk(p, c, sh, saw_nan);
+    if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
+    const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t gthreads = (size_t)gridDim.x * blockDim.x;
+    if (p.coef_t) {
+        for (size_t i = gtid; i < (size_t)2 * p.ncoef; i += gthreads) {
+            const bool second = i >= (size_t)p.ncoef;
+            const size_t j = second ? i - p.ncoef : i;
+            float s, c;
+            sincosf(second ? p.phi[j] : p.theta[j], &s, &c);
+            (second ? p.coef_p : p.coef_t)[j] = make_float2(c, s);
         }
     }
+    if (p.wdec) {
+        if (gtid == 0 && (p.packed[0] != kPackMagic || p.packed[1] != (uint32_t)p.d))
+            set_status(p.status, BFMOE_ERR_INVALID_ARG);
+        const size_t nq = (size_t)p.d * p.d / 8;
+        for (size_t q = gtid; q < nq; q += gthreads) decode_chunk(p.packed, p.d, p.wdec, q);
+    }
+    if ((int)blockIdx.x == p.skip_arrive_block) return;  // test hook: never arrive
+    if (!grid_barrier(p.sync, gridDim.x, p.status, true)) return;
+
+    // ---- phase B: per-expert prefix over chunks
+    {
+        const int warp = (int)(gtid >> 5), lane = threadIdx.x & 31;
+        const int nwarps = (int)(gthreads >> 5);
+        for (int e = warp; e < N; e += nwarps) {
+            int running = 0;
+            for (int c0 = 0; c0 < nchunk; c0 += 32) {
+                const int c = c0 + lane;
+                const int v = c < nchunk ? p.hist[(size_t)c * N + e] : 0;
+                int incl = v;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += o;
+                }
+                if (c < nchunk) p.hist[(size_t)c * N + e] = running + incl - v;
+                running += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) p.total[e] = running;
+        }
+    }
+    if (!grid_barrier(p.sync, 2 * gridDim.x, p.status, true)) return;
+
+    // ---- phase C: bucket offsets, tile list, ranks and scatter
+    int *off = sh;                // [N+1]
+    int *tstart = off + N + 1;    // [N+1]
+    int *cnt = tstart + N + 1;    // [N]
+    int *scratch = cnt + N;       // [blockDim.x]
+    for (int e = threadIdx.x; e < N; e += blockDim.x) {
+        off[e] = p.total[e];
+        if (p.in_tiles) tstart[e] = (off[e] + p.tile_rows - 1) / p.tile_rows;
+    }
+    __syncthreads();
+    const int rsum = block_exclusive_scan(off, off, N, scratch);
+    int ntiles = 0;
+    if (p.in_tiles) ntiles = block_exclusive_scan(tstart, tstart, N, scratch);
+    if (threadIdx.x == 0) {
+        off[N] = rsum;
+        tstart[N] = ntiles;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= N; e += blockDim.x) p.offsets[e] = off[e];
+        if (threadIdx.x == 0 && p.n_in_tiles) *p.n_in_tiles = ntiles;
+    }
+    if (p.in_tiles) {
+        for (int e = (int)gtid; e < N; e += (int)gthreads) {
+            const int n_e = off[e + 1] - off[e];
+            int q = tstart[e];
+            for (int r = 0; r < n_e; r += p.tile_rows, ++q)
+                p.in_tiles[q] = make_int4(e, off[e] + r, min(p.tile_rows, n_e - r), 0);
+        }
+    }
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c = blockIdx.x; c < nchunk; c += gridDim.x) {
+        for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)c * N + e];
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int i0 = c * kRouteChunk * k;
+            const int i1 = min(R, i0 + kRouteChunk * k);
+            for (int c0 = i0; c0 < i1; c0 += 32) {
+                const int i = c0 + lane;
+                const bool valid = i < i1;
+                const int e = valid ? p.topk_idx[i] : -1;
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                const int pos = valid ? cnt[e] + __popc(peers & lt) : 0;
+                __syncwarp();
+                if (valid && (__ffs(peers) - 1) == lane) cnt[e] += __popc(peers);
+                __syncwarp();
+                if (valid) {
+                    p.perm[pos] = i;
+                    if (p.row_pos) p.row_pos[i] = pos;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    pdl_trigger();
 }
+
+__host__ inline size_t route_smem_bytes(int N) { return (size_t)(3 * N + 2 + kRouteThreads) * 4; }
 
 }  // namespace bfmoe

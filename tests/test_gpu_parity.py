@@ -260,3 +260,35 @@ def test_forward_twice_same_workspace_is_deterministic(bf):
     y2, _ = bf.forward(x, lg, 2, packed, th, ph, ws=ws)
     assert bf.sync_status(ws) == bf.OK
     assert torch.equal(y1, y2)
+
+
+# ------------------------------------------------------ failure detection
+# A routing block that never reaches the grid barrier (host-side test hook)
+# makes the others' bounded waits run out: the call must report
+# BFMOE_ERR_TIMEOUT through the status word, not hang or fault, and the
+# context must stay usable.
+
+def test_route_barrier_timeout_reports_status(bf):
+    T, N, k = 2000, 16, 2
+    lg = np.random.default_rng(21).standard_normal((T, N)).astype(np.float32)
+    bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, 0)
+    try:
+        _, _, _, _, ws = bf.route(dev(lg), k)
+        st = bf.sync_status(ws)
+    finally:
+        bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, -1)
+    assert st == bf.ERR_TIMEOUT
+    check_route(bf, lg, k)
+
+
+def test_forward_barrier_timeout_reports_status(bf):
+    inp = wl.make_inputs("headline", T=300)
+    bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, 1)
+    try:
+        _, _, st = run_forward(bf, inp)
+    finally:
+        bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, -1)
+    assert st == bf.ERR_TIMEOUT
+    y, ws, st = run_forward(bf, inp)
+    assert st == bf.OK
+    check_close(y.float().cpu().numpy(), oracle_forward(inp), "after timeout")
