@@ -52,7 +52,8 @@ bfmoe_status check_route_shape(int T, int N, int k)
     return BFMOE_OK;
 }
 
-int route_chunks(int T) { return (T + kRouteChunk - 1) / kRouteChunk; }
+// Rows of the per-block histogram (the routing grid never exceeds it).
+int route_chunks(int) { return kMaxRouteBlocks; }
 
 // Status word and grid-barrier counter share the first 16 bytes of every
 // workspace; one memset clears both.
@@ -219,9 +220,9 @@ bfmoe_status launch_route(RouteParams rp, cudaStream_t st)
     const int sms = device_sms();
     const int occ = occupancy((const void *)k_route, kRouteThreads, smem);
     if (sms <= 0 || occ <= 0) return BFMOE_ERR_CUDA;
-    const int nchunk = route_chunks(rp.T);
-    int grid = std::max(nchunk, 2 * sms);
-    grid = std::min(grid, occ * sms);
+    // one block per SM at most (cheaper grid barriers), never more than the
+    // histogram holds
+    const int grid = std::min(std::min(sms, occ * sms), kMaxRouteBlocks);
     rp.skip_arrive_block = g_skip_arrive_block;
     if (launch(k_route, dim3(grid), dim3(kRouteThreads), smem, st, false, true, rp) != cudaSuccess)
         return BFMOE_ERR_CUDA;
@@ -348,10 +349,10 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
         e = launch(k_combine_sum<T>, dim3((unsigned)((nthreads + 255) / 256)), dim3(256), 0, st, true, false, cb);
         break;
     }
-    case 1: e = launch(k_combine_high<T, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
-    case 2: e = launch(k_combine_high<T, 2>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
-    case 3: e = launch(k_combine_high<T, 3>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
-    default: e = launch(k_combine_high<T, 4>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    case 1: e = launch(k_combine_high<T, 1, 4>, dim3((T_ + 3) / 4), dim3(256), 0, st, true, false, cb); break;
+    case 2: e = launch(k_combine_high<T, 2, 2>, dim3((T_ + 1) / 2), dim3(256), 0, st, true, false, cb); break;
+    case 3: e = launch(k_combine_high<T, 3, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    default: e = launch(k_combine_high<T, 4, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
     }
     if (e != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);

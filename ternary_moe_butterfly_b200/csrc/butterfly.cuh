@@ -22,26 +22,31 @@
 
 namespace bfmoe {
 
-// cos/sin table: float2 {cos a, sin a} per angle, [N][L][d/2].
-template <int G, bool TRANSPOSE>
-__device__ __forceinline__ void bfly_subset(float *row, int base, int s0, const float2 *__restrict__ cf, int half)
+// Pair index of the pair (j, j + 2^s) in stage s: j with bit s deleted.
+__host__ __device__ constexpr int pair_of(int j, int s) { return ((j >> (s + 1)) << s) | (j & ((1 << s) - 1)); }
+
+// One "subset" of a row: the 2^G values whose indices differ only in bits
+// S0..S0+G-1, index base | (m << S0).  Deleting bit s is additive over the
+// disjoint bit sets of base and m << S0, so a rotation's table entry is
+// pair_of(base, s) + pair_of(m << S0, s): one runtime term per stage and a
+// compile-time offset per rotation.  cos/sin table: float2 {cos a, sin a},
+// [L][d/2] for one expert.
+template <int G, int S0, bool TRANSPOSE>
+__device__ __forceinline__ void bfly_subset(float *row, int base, const float2 *__restrict__ cf, int half)
 {
     constexpr int M = 1 << G;
     float v[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) v[m] = row[base + (m << s0)];
+    for (int m = 0; m < M; ++m) v[m] = row[base + (m << S0)];
 #pragma unroll
     for (int q = 0; q < G; ++q) {
         const int ls = TRANSPOSE ? (G - 1 - q) : q;  // local stage
-        const int s = s0 + ls;
-        const int h = 1 << s;
-        const float2 *cs = cf + (size_t)s * half;
+        const int s = S0 + ls;
+        const float2 *cs = cf + (size_t)s * half + pair_of(base, s);
 #pragma unroll
         for (int m = 0; m < M; ++m) {
             if (m & (1 << ls)) continue;
-            const int j = base + (m << s0);
-            const int p = ((j >> (s + 1)) << s) | (j & (h - 1));
-            const float2 c = cs[p];
+            const float2 c = cs[pair_of(m << S0, s)];
             const float sn = TRANSPOSE ? -c.y : c.y;
             const float a = v[m], b = v[m + (1 << ls)];
             v[m] = fmaf(c.x, a, -(sn * b));
@@ -49,45 +54,55 @@ __device__ __forceinline__ void bfly_subset(float *row, int base, int s0, const 
         }
     }
 #pragma unroll
-    for (int m = 0; m < M; ++m) row[base + (m << s0)] = v[m];
+    for (int m = 0; m < M; ++m) row[base + (m << S0)] = v[m];
 }
 
 // Row r uses the table  coef + sexp[r] * estride  (sexp == nullptr: every
 // row uses `coef`, e.g. one expert's table staged in shared memory).
-template <int G, bool TRANSPOSE>
-__device__ void bfly_pass(float *tile, int ld, int rows, int d, int s0, const int *sexp,
-                          const float2 *__restrict__ coef, size_t estride, int nthreads)
+template <int G, int S0, bool TRANSPOSE>
+__device__ void bfly_pass(float *tile, int ld, int rows, int d, const int *sexp, const float2 *__restrict__ coef,
+                          size_t estride, int nthreads)
 {
     const int half = d >> 1;
     const int nsub = d >> G;
-    const int s1 = s0 + G;
+    constexpr int S1 = S0 + G;
     const int items = rows * nsub;
     for (int it = threadIdx.x; it < items; it += nthreads) {
         const int r = it % rows;
         const int sub = it / rows;
-        const int base = ((sub >> s0) << s1) | (sub & ((1 << s0) - 1));
+        const int base = ((sub >> S0) << S1) | (sub & ((1 << S0) - 1));
         const float2 *cf = sexp ? coef + (size_t)sexp[r] * estride : coef;
-        bfly_subset<G, TRANSPOSE>(tile + (size_t)r * ld, base, s0, cf, half);
+        bfly_subset<G, S0, TRANSPOSE>(tile + (size_t)r * ld, base, cf, half);
     }
 }
 
+// Stage split of a butterfly of L stages into passes of at most 5 stages:
+// pass q covers stages [q*L/np, (q+1)*L/np), np = ceil(L/5).
 template <bool TRANSPOSE>
-__device__ __forceinline__ void bfly_pass_g(int g, float *tile, int ld, int rows, int d, int s0, const int *sexp,
-                                            const float2 *coef, size_t estride, int nthreads)
+__device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, float *tile, int ld, int rows, int d,
+                                                   const int *sexp, const float2 *coef, size_t estride)
 {
-    switch (g) {
-    case 1: bfly_pass<1, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
-    case 2: bfly_pass<2, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
-    case 3: bfly_pass<3, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
-    case 4: bfly_pass<4, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
-    default: bfly_pass<5, TRANSPOSE>(tile, ld, rows, d, s0, sexp, coef, estride, nthreads); break;
+    const int nt = blockDim.x;
+#define BFLY_CASE(LL, PP, GG, SS)                                                                     \
+    if (L == LL && pass == PP) {                                                                      \
+        bfly_pass<GG, SS, TRANSPOSE>(tile, ld, rows, d, sexp, coef, estride, nt);                     \
+        return;                                                                                       \
     }
+    BFLY_CASE(6, 0, 3, 0) BFLY_CASE(6, 1, 3, 3)
+    BFLY_CASE(7, 0, 3, 0) BFLY_CASE(7, 1, 4, 3)
+    BFLY_CASE(8, 0, 4, 0) BFLY_CASE(8, 1, 4, 4)
+    BFLY_CASE(9, 0, 4, 0) BFLY_CASE(9, 1, 5, 4)
+    BFLY_CASE(10, 0, 5, 0) BFLY_CASE(10, 1, 5, 5)
+    BFLY_CASE(11, 0, 3, 0) BFLY_CASE(11, 1, 4, 3) BFLY_CASE(11, 2, 4, 7)
+    BFLY_CASE(12, 0, 4, 0) BFLY_CASE(12, 1, 4, 4) BFLY_CASE(12, 2, 4, 8)
+#undef BFLY_CASE
 }
 
 // Apply B (transpose == false) or B^T (transpose == true) to every row r <
 // rows of the tile; row r uses the table of expert sexp[r] (tables of
 // L*d/2 entries, back to back) or, with sexp == nullptr, the single table
-// `coef`.  Must be called by all threads of the block (has __syncthreads).
+// `coef`.  6 <= L <= 12.  Must be called by all threads of the block (has
+// __syncthreads).
 __device__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int *sexp, const float2 *coef,
                           bool transpose)
 {
@@ -95,12 +110,10 @@ __device__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int
     const int npass = (L + 4) / 5;
     for (int q = 0; q < npass; ++q) {
         const int pi = transpose ? (npass - 1 - q) : q;
-        const int s0 = pi * L / npass;
-        const int s1 = (pi + 1) * L / npass;
         if (transpose)
-            bfly_pass_g<true>(s1 - s0, tile, ld, rows, d, s0, sexp, coef, estride, blockDim.x);
+            bfly_pass_dispatch<true>(L, pi, tile, ld, rows, d, sexp, coef, estride);
         else
-            bfly_pass_g<false>(s1 - s0, tile, ld, rows, d, s0, sexp, coef, estride, blockDim.x);
+            bfly_pass_dispatch<false>(L, pi, tile, ld, rows, d, sexp, coef, estride);
         __syncthreads();
     }
 }

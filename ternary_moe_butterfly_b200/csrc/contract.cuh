@@ -15,8 +15,9 @@
 //            through a kStages-deep shared-memory ring;
 //   warp 1   one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of
 //            two TMEM accumulators (double buffered: 2 x BN columns);
-//   warps 2-5  the epilogue: TMEM lane = tile row = thread, so each thread
-//            applies the output-butterfly stages that stay inside the slice
+//   warps 2-9  the epilogue: TMEM lane = tile row = thread, so each thread
+//            (two warps per row, each on half of the columns) applies the
+//            output-butterfly stages that stay inside the slice
 //            (stages 0 .. log2 BN - 1) to its own row, with the row's expert
 //            table, and stores the fp32 result to the row's token-order slot.
 //            Stages 0-4 act inside 32-column blocks (one 32-column TMEM load,
@@ -30,7 +31,7 @@
 
 namespace bfmoe {
 
-constexpr int kContractThreads = 192;
+constexpr int kContractThreads = 320;  // 2 control warps + 8 epilogue warps
 constexpr int kStages = 4;
 
 struct ContractParams {
@@ -56,37 +57,61 @@ __device__ __forceinline__ void rot(float &a, float &b, float2 cs)
     b = fmaf(cs.y, x, cs.x * y);
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// AND of `pred` over the `nthreads` threads of named barrier `id` (a
+// barrier itself): every participant gets the same answer.
+__device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred)
+{
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((int)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // Output-butterfly stages 0 .. log2(BN)-1 of one row held in TMEM columns
-// [tcol, tcol + BN) of this warp's lanes, then store to `out` (if non-null).
+// [tbase, tbase + BN) of this warp's lanes, then store to `out` (if
+// non-null).  Two warps share the row's lanes: `part` (0 or 1) selects which
+// half of the 32-column blocks (pass 1) and of the column groups (pass 2)
+// this warp takes; `bar_id` is a 64-thread named barrier for the pair.
 template <int BN>
 __device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__restrict__ cf, int half,
-                                             float *__restrict__ out)
+                                             float *__restrict__ out, int part, int bar_id)
 {
     constexpr int SIN = BN == 256 ? 8 : (BN == 128 ? 7 : 6);  // log2 BN
     constexpr int G2 = SIN - 5;                              // stages at stride >= 32
     constexpr int M2 = 1 << G2;
+    constexpr int NB = BN / 32;
     // pass 1: stages 0..4 inside each 32-column block
 #pragma unroll 1
-    for (int blk = 0; blk < BN / 32; ++blk) {
+    for (int blk = part * (NB / 2); blk < (part + 1) * (NB / 2); ++blk) {
         float v[32];
         tmem_ld32(tbase + (uint32_t)(blk * 32), v);
 #pragma unroll
         for (int s = 0; s < 5; ++s) {
-            const float2 *cs = cf + (size_t)s * half;
+            const float2 *cs = cf + (size_t)s * half + pair_of(blk * 32, s);
 #pragma unroll
             for (int m = 0; m < 32; ++m) {
                 if (m & (1 << s)) continue;
-                const int jj = blk * 32 + m;
-                const int pl = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
-                rot(v[m], v[m + (1 << s)], __ldg(cs + pl));
+                rot(v[m], v[m + (1 << s)], __ldg(cs + pair_of(m, s)));
             }
         }
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
     }
     tmem_st_wait();
+    named_bar_sync(bar_id, 64);
     // pass 2: stages 5..SIN-1 on columns c + 32 m
 #pragma unroll 1
-    for (int c0 = 0; c0 < 32; c0 += 4) {
+    for (int c0 = part * 16; c0 < part * 16 + 16; c0 += 4) {
         float v[4][M2];
 #pragma unroll
         for (int m = 0; m < M2; ++m)
@@ -95,15 +120,13 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__res
 #pragma unroll
         for (int ls = 0; ls < G2; ++ls) {
             const int s = 5 + ls;
-            const float2 *cs = cf + (size_t)s * half;
+            const float2 *cs = cf + (size_t)s * half + pair_of(c0, s);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
                 for (int m = 0; m < M2; ++m) {
                     if (m & (1 << ls)) continue;
-                    const int jj = c0 + q + 32 * m;
-                    const int pl = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
-                    rot(v[q][m], v[q][m + (1 << ls)], __ldg(cs + pl));
+                    rot(v[q][m], v[q][m + (1 << ls)], __ldg(cs + pair_of(q + 32 * m, s)));
                 }
             }
         }
@@ -143,7 +166,7 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], 8);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -221,13 +244,18 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             if (!mbar_wait(drain, 0)) set_status(p.status, BFMOE_ERR_TIMEOUT);
         }
     } else {
-        // epilogue warps 2..5 own TMEM lanes 32*(warp % 4) .. +31
+        // epilogue warps 2..9: warp w owns TMEM lanes 32*(w % 4) .. +31 and
+        // half of the row's columns (part = (w - 2) / 4)
         const int lane_base = (warp & 3) * 32;
+        const int part = (warp - 2) >> 2;
+        const int bar_id = 1 + (warp & 3);
         int li = 0;
         for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++li) {
             const int b = li & 1;
             bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
-            ok = __all_sync(0xffffffffu, ok);
+            // both warps sharing these lanes take the same branch (they meet
+            // at a named barrier inside epilogue_row)
+            ok = bar_red_and(bar_id, 64, ok);
             if (!ok) {
                 if (lane == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
                 break;
@@ -243,7 +271,7 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             }
             const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)nh * (BN / 2);
             float *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
-            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, half, out);
+            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, half, out, part, bar_id);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);

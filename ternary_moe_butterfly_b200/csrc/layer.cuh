@@ -177,13 +177,32 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
             stok[threadIdx.x] = t;
         }
         __syncthreads();
-        for (int q = warp; q < nr; q += nw) {
-            const int t = stok[q];
-            float *dst = tile + (size_t)q * ld;
-            if (t >= 0)
-                warp_load_row<T>(x + (size_t)t * d, dst, d, lane);
-            else
-                for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
+        // gather: lane = tile row, warp = 16-byte column chunk, so the scalar
+        // shared-memory stores of a warp hit 32 distinct banks
+        {
+            const int t = lane < nr ? stok[lane] : -1;
+            constexpr int VPC = 16 / sizeof(T);  // values per 16-byte chunk
+            for (int c = warp; c < d / VPC; c += nw) {
+                if (lane >= nr) continue;
+                float f[8];
+                if (t >= 0) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c);
+                    if (VPC == 8) {
+                        unpack_bf16x8(u, f);
+                    } else {
+                        f[0] = __uint_as_float(u.x);
+                        f[1] = __uint_as_float(u.y);
+                        f[2] = __uint_as_float(u.z);
+                        f[3] = __uint_as_float(u.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] = 0.0f;
+                }
+                float *dst = tile + (size_t)lane * ld + c * VPC;
+#pragma unroll
+                for (int i = 0; i < VPC; ++i) dst[i] = f[i];
+            }
         }
         __syncthreads();
         bfly_tile(tile, ld, nr, d, L, nullptr, SMEM_COEF ? sc : gtab, /*transpose=*/true);
@@ -227,52 +246,66 @@ struct CombineParams {
     void *y;
 };
 
-// HS = L - s_lo > 0 high stages: one token per block, 256 threads; thread c
-// owns columns c + 256 m (m < 2^HS), which the stages s_lo..L-1 mix.
-template <typename T, int HS>
+// HS = L - s_lo > 0 high stages: TPB tokens per block, 256 threads; thread c
+// owns columns c + 256 m (m < 2^HS) of each token, which the stages
+// s_lo..L-1 mix.  All slot and table loads of a token are issued before any
+// arithmetic so that each thread keeps many loads in flight.
+template <typename T, int HS, int TPB>
 __global__ void __launch_bounds__(256) k_combine_high(CombineParams p)
 {
     pdl_wait();
     pdl_trigger();
     constexpr int G = 1 << HS;
-    const int t = blockIdx.x;
-    if (t >= p.T) return;
     const int c = threadIdx.x;
     const int d = p.d, half = d >> 1;
-    float acc[G];
-#pragma unroll
-    for (int m = 0; m < G; ++m) acc[m] = 0.0f;
-    for (int j = 0; j < p.k; ++j) {
-        const int i = t * p.k + j;
-        const int e = min(max(p.topk_idx[i], 0), p.N - 1);
-        const float g = p.gates[i];
-        const float *row = p.slot + (size_t)i * d;
-        float v[G];
-#pragma unroll
-        for (int m = 0; m < G; ++m) v[m] = row[c + 256 * m];
-        const float2 *cf = p.coef_p + (size_t)e * p.L * half;
-#pragma unroll
-        for (int ls = 0; ls < HS; ++ls) {
-            const int s = p.s_lo + ls;
-            const float2 *cs = cf + (size_t)s * half;
-#pragma unroll
-            for (int m = 0; m < G; ++m) {
-                if (m & (1 << ls)) continue;
-                const int jj = c + 256 * m;
-                const int pp = ((jj >> (s + 1)) << s) | (jj & ((1 << s) - 1));
-                const float2 cs2 = __ldg(cs + pp);
-                const float a = v[m], b = v[m + (1 << ls)];
-                v[m] = fmaf(cs2.x, a, -(cs2.y * b));
-                v[m + (1 << ls)] = fmaf(cs2.y, a, cs2.x * b);
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < G; ++m) acc[m] = fmaf(g, v[m], acc[m]);
-    }
     const float alpha = __uint_as_float(__ldg(p.packed + 2));
-    T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d;
+#pragma unroll 1
+    for (int tt = 0; tt < TPB; ++tt) {
+        const int t = blockIdx.x * TPB + tt;
+        if (t >= p.T) return;
+        float acc[G];
 #pragma unroll
-    for (int m = 0; m < G; ++m) store1(y + c + 256 * m, alpha * acc[m]);
+        for (int m = 0; m < G; ++m) acc[m] = 0.0f;
+#pragma unroll 1
+        for (int j = 0; j < p.k; ++j) {
+            const int i = t * p.k + j;
+            const int e = min(max(p.topk_idx[i], 0), p.N - 1);
+            const float g = p.gates[i];
+            const float *row = p.slot + (size_t)i * d;
+            float v[G];
+            float2 cs[HS][G / 2];
+            const float2 *cf = p.coef_p + (size_t)e * p.L * half;
+#pragma unroll
+            for (int m = 0; m < G; ++m) v[m] = row[c + 256 * m];
+#pragma unroll
+            for (int ls = 0; ls < HS; ++ls) {
+                const int s = p.s_lo + ls;
+                int q = 0;
+#pragma unroll
+                for (int m = 0; m < G; ++m) {
+                    if (m & (1 << ls)) continue;
+                    cs[ls][q++] = __ldg(cf + (size_t)s * half + pair_of(c + 256 * m, s));
+                }
+            }
+#pragma unroll
+            for (int ls = 0; ls < HS; ++ls) {
+                int q = 0;
+#pragma unroll
+                for (int m = 0; m < G; ++m) {
+                    if (m & (1 << ls)) continue;
+                    const float2 w = cs[ls][q++];
+                    const float a = v[m], b = v[m + (1 << ls)];
+                    v[m] = fmaf(w.x, a, -(w.y * b));
+                    v[m + (1 << ls)] = fmaf(w.y, a, w.x * b);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < G; ++m) acc[m] = fmaf(g, v[m], acc[m]);
+        }
+        T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d;
+#pragma unroll
+        for (int m = 0; m < G; ++m) store1(y + c + 256 * m, alpha * acc[m]);
+    }
 }
 
 // No stage left (d <= 256): 8 columns per thread.

@@ -9,13 +9,14 @@
 //
 // Phases, separated by two bounded grid barriers (all blocks are
 // co-resident: the kernel is launched cooperatively):
-//   A  one warp per token selects the top-k; each 64-token chunk counts its
-//      rows per expert (hist[chunk][e]).  While the routing runs, the same
+//   A  each block takes a contiguous token range; batches of its tokens'
+//      logits are staged in shared memory and one warp per token selects
+//      the top-k; the block counts its rows per expert (hist[block][e]).  While the routing runs, the same
 //      blocks also turn the butterfly angles into {cos, sin} tables and
 //      decode the packed ternary base into the tensor-core operand layout
 //      (forward only).
-//   B  one warp per expert scans hist[.][e] over the chunks (exclusive
-//      prefix per chunk, total per expert).
+//   B  one warp per expert scans hist[.][e] over the blocks (exclusive
+//      prefix per block, total per expert).
 //   C  every block scans the expert totals into bucket offsets, then ranks
 //      the rows of its chunks inside their buckets (warp match + popcount)
 //      and scatters perm / row_pos; the blocks also write the list of
@@ -27,8 +28,8 @@
 namespace bfmoe {
 
 constexpr int kRouteThreads = 256;
-constexpr int kRouteChunk = 64;  // tokens per chunk: 8 warps x 8 tokens
 constexpr int kMaxK = 8;
+constexpr int kMaxRouteBlocks = 512;  // capacity of the per-block histogram
 constexpr uint32_t kPackMagic = 0x32574642u;  // "BFW2"
 
 __host__ __device__ constexpr int gemm_bn(int d) { return d < 256 ? d : 256; }
@@ -42,7 +43,7 @@ struct RouteParams {
     int32_t *perm;       // [T*k]
     int32_t *row_pos;    // [T*k] or null
     int32_t *offsets;    // [N+1]
-    int32_t *hist;       // [nchunk][N] -> per-chunk bucket bases
+    int32_t *hist;       // [gridDim][N] -> per-block bucket bases
     int32_t *total;      // [N]
     uint32_t *sync;      // grid barrier counter, zero at launch
     uint32_t *status;
@@ -59,6 +60,13 @@ struct RouteParams {
     int32_t *n_in_tiles;
     int tile_rows;
 };
+
+// Tokens staged per batch: up to 64, at most 32 KB of logits.
+__host__ __device__ inline int route_batch_tokens(int N)
+{
+    const int b = (32 * 1024 / 4) / N;
+    return b < 1 ? 1 : (b > 64 ? 64 : b);
+}
 
 // (va, a) ranks before (vb, b)?  NaN has been mapped to -inf by the caller.
 __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b)
@@ -92,80 +100,105 @@ __device__ bool grid_barrier(uint32_t *ctr, uint32_t target, uint32_t *status, b
     return ok != 0;
 }
 
-// Top-k, gates and the chunk histogram for tokens [c*64, c*64+64).
-__device__ void topk_chunk(const RouteParams &p, int c, int *sh_hist, bool &saw_nan)
+// Top-k and gates of one token whose N logits are in shared memory (NaN
+// already replaced by -inf); one warp.  Lane 0 writes the results and counts
+// the token's rows in the block histogram.
+__device__ __forceinline__ void topk_token(const RouteParams &p, int t, const float *l, int *sh_hist)
 {
     const int N = p.N, k = p.k;
-    for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tok0 = c * kRouteChunk + warp * (kRouteChunk / 8);
-    for (int q = 0; q < kRouteChunk / 8; ++q) {
-        const int t = tok0 + q;
-        if (t >= p.T) break;
-        const float *l = p.logits + (size_t)t * N;
-        int sel[kMaxK];
-        float val[kMaxK];
+    const int lane = threadIdx.x & 31;
+    int sel[kMaxK];
+    float val[kMaxK];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
-            if (j >= k) break;
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-            for (int e = lane; e < N; e += 32) {
-                bool taken = false;
+    for (int j = 0; j < kMaxK; ++j) {
+        if (j >= k) break;
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+        for (int e = lane; e < N; e += 32) {
+            bool taken = false;
 #pragma unroll
-                for (int jj = 0; jj < kMaxK; ++jj)
-                    if (jj < j) taken |= (sel[jj] == e);
-                if (taken) continue;
-                float v = __ldg(l + e);
-                if (v != v) {
-                    saw_nan = true;
-                    v = -INFINITY;
-                }
-                if (be == 0x7fffffff || ranks_before(v, e, bv, be)) {
-                    bv = v;
-                    be = e;
-                }
+            for (int jj = 0; jj < kMaxK; ++jj)
+                if (jj < j) taken |= (sel[jj] == e);
+            if (taken) continue;
+            const float v = l[e];
+            if (be == 0x7fffffff || ranks_before(v, e, bv, be)) {
+                bv = v;
+                be = e;
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || ranks_before(ov, oe, bv, be))) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            sel[j] = be;
-            val[j] = bv;
         }
-        if (lane == 0) {
-            float g[kMaxK];
-            const float m = val[0];
-            if (m == INFINITY) {
-                int cnt = 0;
-                for (int j = 0; j < k; ++j) cnt += (val[j] == INFINITY);
-                for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)cnt : 0.0f;
-            } else if (m == -INFINITY) {
-                for (int j = 0; j < k; ++j) g[j] = 1.0f / (float)k;
-            } else {
-                float z = 0.0f;
-                for (int j = 0; j < k; ++j) {
-                    g[j] = expf(val[j] - m);
-                    z += g[j];
-                }
-                const float rz = 1.0f / z;
-                for (int j = 0; j < k; ++j) g[j] *= rz;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (oe != 0x7fffffff && (be == 0x7fffffff || ranks_before(ov, oe, bv, be))) {
+                bv = ov;
+                be = oe;
             }
+        }
+        sel[j] = be;
+        val[j] = bv;
+    }
+    if (lane == 0) {
+        float g[kMaxK];
+        const float m = val[0];
+        if (m == INFINITY) {
+            int cnt = 0;
+            for (int j = 0; j < k; ++j) cnt += (val[j] == INFINITY);
+            for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)cnt : 0.0f;
+        } else if (m == -INFINITY) {
+            for (int j = 0; j < k; ++j) g[j] = 1.0f / (float)k;
+        } else {
+            float z = 0.0f;
             for (int j = 0; j < k; ++j) {
-                p.topk_idx[(size_t)t * k + j] = sel[j];
-                p.gates[(size_t)t * k + j] = g[j];
-                atomicAdd(&sh_hist[sel[j]], 1);
+                g[j] = expf(val[j] - m);
+                z += g[j];
             }
+            const float rz = 1.0f / z;
+            for (int j = 0; j < k; ++j) g[j] *= rz;
+        }
+        for (int j = 0; j < k; ++j) {
+            p.topk_idx[(size_t)t * k + j] = sel[j];
+            p.gates[(size_t)t * k + j] = g[j];
+            atomicAdd(&sh_hist[sel[j]], 1);
         }
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)c * N + e] = sh_hist[e];
+}
+
+// Top-k, gates and the histogram of the block's token range [t0, t1):
+// batches of tokens are staged in shared memory with coalesced 16-byte loads
+// (one memory latency per batch), then one warp per token selects.
+__device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, float *sh_logits, int batch,
+                           bool &saw_nan)
+{
+    const int N = p.N;
+    for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int b0 = t0; b0 < t1; b0 += batch) {
+        const int nb = min(batch, t1 - b0);
+        const size_t nval = (size_t)nb * N;
+        const float *src = p.logits + (size_t)b0 * N;
+        __syncthreads();
+        if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(src);
+            float4 *d4 = reinterpret_cast<float4 *>(sh_logits);
+            for (size_t q = threadIdx.x; q < nval / 4; q += blockDim.x) {
+                float4 v = __ldg(s4 + q);
+                if (v.x != v.x) { saw_nan = true; v.x = -INFINITY; }
+                if (v.y != v.y) { saw_nan = true; v.y = -INFINITY; }
+                if (v.z != v.z) { saw_nan = true; v.z = -INFINITY; }
+                if (v.w != v.w) { saw_nan = true; v.w = -INFINITY; }
+                d4[q] = v;
+            }
+        } else {
+            for (size_t q = threadIdx.x; q < nval; q += blockDim.x) {
+                float v = __ldg(src + q);
+                if (v != v) { saw_nan = true; v = -INFINITY; }
+                sh_logits[q] = v;
+            }
+        }
+        __syncthreads();
+        for (int q = warp; q < nb; q += nw) topk_token(p, b0 + q, sh_logits + (size_t)q * N, sh_hist);
+    }
     __syncthreads();
 }
 
@@ -229,12 +262,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
 {
     extern __shared__ int sh[];  // phase A: hist[N]; phase C: off[N+1], tstart[N+1], cnt[N], scratch[256]
     const int N = p.N, k = p.k;
-    const int nchunk = (p.T + kRouteChunk - 1) / kRouteChunk;
-    const int R = p.T * k;
+    const int nchunk = gridDim.x;  // one histogram row per block
 
-    // ---- phase A: top-k and chunk histograms, plus the prep work
+    // ---- phase A: top-k over this block's token range, plus the prep work
+    float *sh_logits = reinterpret_cast<float *>(sh + N);
+    const int batch = route_batch_tokens(N);
     bool saw_nan = false;
-    for (int c = blockIdx.x; c < nchunk; c += gridDim.x) topk_chunk(p, c, sh, saw_nan);
+    const int tpb = (p.T + gridDim.x - 1) / gridDim.x;  // tokens per block
+    const int t0 = min(p.T, (int)blockIdx.x * tpb), t1 = min(p.T, t0 + tpb);
+    topk_range(p, t0, t1, sh, sh_logits, batch, saw_nan);
+    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)blockIdx.x * N + e] = sh[e];
     if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t gthreads = (size_t)gridDim.x * blockDim.x;
@@ -311,32 +348,33 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     }
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
-    for (int c = blockIdx.x; c < nchunk; c += gridDim.x) {
-        for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)c * N + e];
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            const int i0 = c * kRouteChunk * k;
-            const int i1 = min(R, i0 + kRouteChunk * k);
-            for (int c0 = i0; c0 < i1; c0 += 32) {
-                const int i = c0 + lane;
-                const bool valid = i < i1;
-                const int e = valid ? p.topk_idx[i] : -1;
-                const unsigned peers = __match_any_sync(0xffffffffu, e);
-                const int pos = valid ? cnt[e] + __popc(peers & lt) : 0;
-                __syncwarp();
-                if (valid && (__ffs(peers) - 1) == lane) cnt[e] += __popc(peers);
-                __syncwarp();
-                if (valid) {
-                    p.perm[pos] = i;
-                    if (p.row_pos) p.row_pos[i] = pos;
-                }
+    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)blockIdx.x * N + e];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int i0 = t0 * k, i1 = t1 * k;
+        for (int c0 = i0; c0 < i1; c0 += 32) {
+            const int i = c0 + lane;
+            const bool valid = i < i1;
+            const int e = valid ? p.topk_idx[i] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int pos = valid ? cnt[e] + __popc(peers & lt) : 0;
+            __syncwarp();
+            if (valid && (__ffs(peers) - 1) == lane) cnt[e] += __popc(peers);
+            __syncwarp();
+            if (valid) {
+                p.perm[pos] = i;
+                if (p.row_pos) p.row_pos[i] = pos;
             }
         }
-        __syncthreads();
     }
     pdl_trigger();
 }
 
-__host__ inline size_t route_smem_bytes(int N) { return (size_t)(3 * N + 2 + kRouteThreads) * 4; }
+__host__ inline size_t route_smem_bytes(int N)
+{
+    const size_t a = (size_t)N * 4 + (size_t)route_batch_tokens(N) * N * 4;  // phase A
+    const size_t c = (size_t)(3 * N + 2 + kRouteThreads) * 4;              // phase C
+    return a > c ? a : c;
+}
 
 }  // namespace bfmoe
