@@ -579,6 +579,20 @@ bfmoe_status bfmoe_forward_profile(const void *x, bfmoe_dtype dt, int T, int d, 
     return s;
 }
 
+#ifdef BFMOE_TRACE_PHASES
+// Copy the phase trace (4 kernels x 1024 blocks x 16 slots of u64) to host.
+BFMOE_API int bfmoe_trace_read(unsigned long long *host, int clear)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) return BFMOE_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(host, g_bfmoe_trace, sizeof(g_bfmoe_trace)) != cudaSuccess) return BFMOE_ERR_CUDA;
+    if (clear) {
+        static unsigned long long zeros[4][kTraceBlocks][kTraceSlots];
+        if (cudaMemcpyToSymbol(g_bfmoe_trace, zeros, sizeof(zeros)) != cudaSuccess) return BFMOE_ERR_CUDA;
+    }
+    return BFMOE_OK;
+}
+#endif
+
 const char *bfmoe_stage_name(int i) { return (i >= 0 && i < kNumStages) ? kStageNames[i] : nullptr; }
 
 bfmoe_status bfmoe_sync_status(void *ws, void *stream)

@@ -33,6 +33,24 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------- phase trace --
+// Built with -DBFMOE_TRACE_PHASES, kernels record %globaltimer at phase
+// boundaries: g_bfmoe_trace[kernel][block][slot] (read back with
+// bfmoe_trace_read).  Without the flag the macro compiles to nothing.
+#ifdef BFMOE_TRACE_PHASES
+constexpr int kTraceBlocks = 1024, kTraceSlots = 16;
+__device__ unsigned long long g_bfmoe_trace[4][kTraceBlocks][kTraceSlots];
+#define BFMOE_TRACE(kernel, cond, slot)                                                     \
+    do {                                                                                    \
+        if ((cond) && blockIdx.x < kTraceBlocks)                                            \
+            ::bfmoe::g_bfmoe_trace[(kernel)][blockIdx.x][(slot)] = ::bfmoe::globaltimer_ns(); \
+    } while (0)
+#else
+#define BFMOE_TRACE(kernel, cond, slot) \
+    do {                                \
+    } while (0)
+#endif
+
 // ------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)

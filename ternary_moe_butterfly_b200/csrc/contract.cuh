@@ -32,7 +32,15 @@
 namespace bfmoe {
 
 constexpr int kContractThreads = 320;  // 2 control warps + 8 epilogue warps
-constexpr int kStages = 4;
+constexpr int kStages = 3;
+
+// log2 of the output slice width: the output-butterfly stages the epilogue
+// applies.
+__host__ __device__ constexpr int slice_stages(int BN) { return BN == 256 ? 8 : (BN == 128 ? 7 : 6); }
+
+// Shared-memory cos/sin tables staged per pair of epilogue warps: two
+// experts x slice_stages(BN) stages x BN/2 pairs.
+__host__ __device__ constexpr int pair_table_floats2(int BN) { return 2 * slice_stages(BN) * (BN / 2); }
 
 struct ContractParams {
     const __half *a_blocks;   // [Rp/128][d/64] blocks of 128 x 64
@@ -84,10 +92,10 @@ __device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred)
 // half of the 32-column blocks (pass 1) and of the column groups (pass 2)
 // this warp takes; `bar_id` is a 64-thread named barrier for the pair.
 template <int BN>
-__device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__restrict__ cf, int half,
+__device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__restrict__ cf, int cstride,
                                              float *__restrict__ out, int part, int bar_id)
 {
-    constexpr int SIN = BN == 256 ? 8 : (BN == 128 ? 7 : 6);  // log2 BN
+    constexpr int SIN = slice_stages(BN);
     constexpr int G2 = SIN - 5;                              // stages at stride >= 32
     constexpr int M2 = 1 << G2;
     constexpr int NB = BN / 32;
@@ -98,11 +106,11 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__res
         tmem_ld32(tbase + (uint32_t)(blk * 32), v);
 #pragma unroll
         for (int s = 0; s < 5; ++s) {
-            const float2 *cs = cf + (size_t)s * half + pair_of(blk * 32, s);
+            const float2 *cs = cf + s * cstride + pair_of(blk * 32, s);
 #pragma unroll
             for (int m = 0; m < 32; ++m) {
                 if (m & (1 << s)) continue;
-                rot(v[m], v[m + (1 << s)], __ldg(cs + pair_of(m, s)));
+                rot(v[m], v[m + (1 << s)], cs[pair_of(m, s)]);
             }
         }
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
@@ -120,13 +128,13 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__res
 #pragma unroll
         for (int ls = 0; ls < G2; ++ls) {
             const int s = 5 + ls;
-            const float2 *cs = cf + (size_t)s * half + pair_of(c0, s);
+            const float2 *cs = cf + s * cstride + pair_of(c0, s);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
                 for (int m = 0; m < M2; ++m) {
                     if (m & (1 << ls)) continue;
-                    rot(v[q][m], v[q][m + (1 << ls)], __ldg(cs + pair_of(q + 32 * m, s)));
+                    rot(v[q][m], v[q][m + (1 << ls)], cs[pair_of(q + 32 * m, s)]);
                 }
             }
         }
@@ -157,8 +165,10 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
     uint64_t *tfull = bars + 2 * kStages, *tempty = tfull + 2, *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile uint32_t *abort_flag = tmem_slot + 1;
+    float2 *tables = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(bars) + 256);  // [4 pairs][...]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BFMOE_TRACE(2, threadIdx.x == 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -177,8 +187,10 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    BFMOE_TRACE(2, threadIdx.x == 0, 1);
     pdl_wait();  // the A blocks come from the input-butterfly kernel
     pdl_trigger();
+    BFMOE_TRACE(2, threadIdx.x == 0, 2);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -195,6 +207,7 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
                         *abort_flag = 1;
                         break;
                     }
+                    BFMOE_TRACE(2, it == 0, 3);
                     mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
                     bulk_g2s(sA + (size_t)s * a_bytes, a_src + (size_t)kc * (kBM * kBK), a_bytes, &full[s]);
                     bulk_g2s(sB + (size_t)s * b_bytes, b_src + (size_t)kc * ((size_t)BN * kBK), b_bytes, &full[s]);
@@ -227,6 +240,8 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
                         break;
                     }
                     tc_fence_after();
+                    BFMOE_TRACE(2, it == 0, 4);
+                    BFMOE_TRACE(2, it == KC - 1, 5);
                     const uint32_t a0 = smem_addr(sA + (size_t)s * a_bytes), b0 = smem_addr(sB + (size_t)s * b_bytes);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -249,18 +264,13 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
         const int lane_base = (warp & 3) * 32;
         const int part = (warp - 2) >> 2;
         const int bar_id = 1 + (warp & 3);
+        constexpr int SIN = slice_stages(BN);
+        constexpr int HB = BN / 2;  // pairs per stage inside the slice
+        float2 *ptab = tables + (size_t)(warp & 3) * pair_table_floats2(BN);
+        const int pt = (part << 5) | lane;  // thread index inside the warp pair
         int li = 0;
         for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++li) {
             const int b = li & 1;
-            bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
-            // both warps sharing these lanes take the same branch (they meet
-            // at a named barrier inside epilogue_row)
-            ok = bar_red_and(bar_id, 64, ok);
-            if (!ok) {
-                if (lane == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
-                break;
-            }
-            tc_fence_after();
             const int mt = u / NH, nh = u % NH;
             const int r = mt * kBM + lane_base + lane;
             int i = -1, e = 0;
@@ -269,9 +279,40 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
                 if (i < 0 || i >= p.R) i = -1;
                 else e = min(max(p.topk_idx[i], 0), p.N - 1);
             }
-            const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)nh * (BN / 2);
+            // the rows are in bucket order: stage the tables of the first and
+            // last row's experts for this slice while the MMA runs
+            const int ea = __shfl_sync(0xffffffffu, e, 0), eb = __shfl_sync(0xffffffffu, e, 31);
+            named_bar_sync(bar_id, 64);  // the pair is done with the previous unit's tables
+            for (int q = pt; q < 2 * SIN * (HB / 2); q += 64) {
+                const int t = q / (SIN * (HB / 2)), rem = q % (SIN * (HB / 2));
+                const int sidx = rem / (HB / 2), w = rem % (HB / 2);
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    p.coef_p + ((size_t)(t ? eb : ea) * p.L + sidx) * half + (size_t)nh * HB);
+                reinterpret_cast<float4 *>(ptab + (size_t)(t * SIN + sidx) * HB)[w] = __ldg(src + w);
+            }
+            bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
+            // both warps sharing these lanes take the same branch (they meet
+            // at named barriers inside epilogue_row); the barrier also makes
+            // the staged tables visible to the pair
+            ok = bar_red_and(bar_id, 64, ok);
+            if (!ok) {
+                if (lane == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
+                break;
+            }
+            tc_fence_after();
+            BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 6);
+            const float2 *cf;
+            int cstride;
+            if (e == ea || e == eb) {
+                cf = ptab + (e == ea ? 0 : SIN * HB);
+                cstride = HB;
+            } else {  // a third expert inside 32 rows: read its table from global memory
+                cf = p.coef_p + (size_t)e * p.L * half + (size_t)nh * HB;
+                cstride = half;
+            }
             float *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
-            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, half, out, part, bar_id);
+            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, cstride, out, part, bar_id);
+            BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 7);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);
@@ -280,12 +321,14 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+    BFMOE_TRACE(2, threadIdx.x == 0, 8);
 }
 
 __host__ inline size_t contract_smem_bytes(int d)
 {
     const int BN = gemm_bn(d);
-    return 1024 + (size_t)kStages * (kBM * kBK * 2 + (size_t)BN * kBK * 2) + (2 * kStages + 5) * 8 + 16;
+    return 1024 + (size_t)kStages * (kBM * kBK * 2 + (size_t)BN * kBK * 2) + 256 +
+           (size_t)4 * pair_table_floats2(BN) * 8;
 }
 
 }  // namespace bfmoe

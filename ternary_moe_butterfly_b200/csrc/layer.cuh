@@ -147,8 +147,10 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
     float2 *sc = reinterpret_cast<float2 *>(smem_f);  // [tab] when SMEM_COEF
     float *tile = smem_f + (SMEM_COEF ? 2 * tab : 0);
     int *stok = reinterpret_cast<int *>(tile + (size_t)RT * ld);
+    BFMOE_TRACE(1, threadIdx.x == 0, 0);
     pdl_wait();
     pdl_trigger();
+    BFMOE_TRACE(1, threadIdx.x == 0, 1);
     // a routing that gave up (timeout) leaves the list unspecified: clamp it
     const int ntiles = min(max(*p.n_tiles, 0), p.max_tiles);
     const T *x = reinterpret_cast<const T *>(p.x);
@@ -178,34 +180,45 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
         }
         __syncthreads();
         // gather: lane = tile row, warp = 16-byte column chunk, so the scalar
-        // shared-memory stores of a warp hit 32 distinct banks
+        // shared-memory stores of a warp hit 32 distinct banks; each lane
+        // issues a batch of 8 loads before converting any of them
         {
             const int t = lane < nr ? stok[lane] : -1;
             constexpr int VPC = 16 / sizeof(T);  // values per 16-byte chunk
-            for (int c = warp; c < d / VPC; c += nw) {
-                if (lane >= nr) continue;
-                float f[8];
-                if (t >= 0) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d) + c);
-                    if (VPC == 8) {
-                        unpack_bf16x8(u, f);
-                    } else {
-                        f[0] = __uint_as_float(u.x);
-                        f[1] = __uint_as_float(u.y);
-                        f[2] = __uint_as_float(u.z);
-                        f[3] = __uint_as_float(u.w);
-                    }
-                } else {
+            const int nchunk = d / VPC;
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(t >= 0 ? t : 0) * d);
+            float *dst = tile + (size_t)lane * ld;
+            for (int c0 = warp; c0 < nchunk; c0 += 8 * nw) {
+                uint4 u[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] = 0.0f;
+                for (int q = 0; q < 8; ++q) {
+                    const int c = c0 + q * nw;
+                    u[q] = (t >= 0 && c < nchunk) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
                 }
-                float *dst = tile + (size_t)lane * ld + c * VPC;
+                if (lane < nr) {
 #pragma unroll
-                for (int i = 0; i < VPC; ++i) dst[i] = f[i];
+                    for (int q = 0; q < 8; ++q) {
+                        const int c = c0 + q * nw;
+                        if (c >= nchunk) break;
+                        float f[8];
+                        if (VPC == 8) {
+                            unpack_bf16x8(u[q], f);
+                        } else {
+                            f[0] = __uint_as_float(u[q].x);
+                            f[1] = __uint_as_float(u[q].y);
+                            f[2] = __uint_as_float(u[q].z);
+                            f[3] = __uint_as_float(u[q].w);
+                        }
+#pragma unroll
+                        for (int i = 0; i < VPC; ++i) dst[c * VPC + i] = f[i];
+                    }
+                }
             }
         }
         __syncthreads();
+        BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 3);
         bfly_tile(tile, ld, nr, d, L, nullptr, SMEM_COEF ? sc : gtab, /*transpose=*/true);
+        BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 4);
         bool overflow = false;
         const int nch = nr * (d / 8);
         for (int q = threadIdx.x; q < nch; q += blockDim.x) {
@@ -223,6 +236,7 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
         if (overflow) set_status(p.status, BFMOE_ERR_NONFINITE);
         __syncthreads();
     }
+    BFMOE_TRACE(1, threadIdx.x == 0, 2);
 }
 
 __host__ inline size_t expert_in_smem_bytes(int d, int L, bool smem_coef)
@@ -253,8 +267,10 @@ struct CombineParams {
 template <typename T, int HS, int TPB>
 __global__ void __launch_bounds__(256) k_combine_high(CombineParams p)
 {
+    BFMOE_TRACE(3, threadIdx.x == 0, 0);
     pdl_wait();
     pdl_trigger();
+    BFMOE_TRACE(3, threadIdx.x == 0, 1);
     constexpr int G = 1 << HS;
     const int c = threadIdx.x;
     const int d = p.d, half = d >> 1;

@@ -10,15 +10,16 @@
 // Phases, separated by two bounded grid barriers (all blocks are
 // co-resident: the kernel is launched cooperatively):
 //   A  each block takes a contiguous token range; batches of its tokens'
-//      logits are staged in shared memory and one warp per token selects
-//      the top-k; the block counts its rows per expert (hist[block][e]).  While the routing runs, the same
-//      blocks also turn the butterfly angles into {cos, sin} tables and
-//      decode the packed ternary base into the tensor-core operand layout
-//      (forward only).
+//      logits are staged in shared memory and one thread (one warp beyond
+//      256 experts) per token selects the top-k; the block counts its rows
+//      per expert (hist[block][e]).  Between arriving at the first barrier
+//      and waiting on it, the blocks turn the butterfly angles into
+//      {cos, sin} tables and decode the packed ternary base into the
+//      tensor-core operand layout (forward only).
 //   B  one warp per expert scans hist[.][e] over the blocks (exclusive
 //      prefix per block, total per expert).
 //   C  every block scans the expert totals into bucket offsets, then ranks
-//      the rows of its chunks inside their buckets (warp match + popcount)
+//      the rows of its tokens inside their buckets (warp match + popcount)
 //      and scatters perm / row_pos; the blocks also write the list of
 //      single-expert row tiles that the input-butterfly kernel walks.
 #pragma once
@@ -61,11 +62,15 @@ struct RouteParams {
     int tile_rows;
 };
 
-// Tokens staged per batch: up to 64, at most 32 KB of logits.
+// Up to this many experts one thread selects a token's top-k.
+constexpr int kThreadTopkMaxN = 256;
+
+// Tokens staged per batch: one per thread (at most 256), at most ~40 KB of
+// logits.
 __host__ __device__ inline int route_batch_tokens(int N)
 {
-    const int b = (32 * 1024 / 4) / N;
-    return b < 1 ? 1 : (b > 64 ? 64 : b);
+    const int b = (40 * 1024 / 4) / (N + 1);
+    return b < 1 ? 1 : (b > 256 ? 256 : b);
 }
 
 // (va, a) ranks before (vb, b)?  NaN has been mapped to -inf by the caller.
@@ -74,16 +79,23 @@ __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b)
     return va > vb || (va == vb && a < b);
 }
 
-// Bounded grid-wide barrier on a monotonically increasing counter.  Returns
-// false (block-uniformly) if the other blocks did not arrive in time.
-__device__ bool grid_barrier(uint32_t *ctr, uint32_t target, uint32_t *status, bool arrive)
+// Split-phase grid-wide barrier on a monotonically increasing counter:
+// arrive publishes the block's earlier writes; wait (bounded) returns false,
+// block-uniformly, if the other blocks did not arrive in time.
+__device__ __forceinline__ void grid_arrive(uint32_t *ctr)
 {
-    __shared__ int ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        ok = 1;
         __threadfence();
-        if (arrive) atomicAdd(ctr, 1u);
+        atomicAdd(ctr, 1u);
+    }
+}
+
+__device__ bool grid_wait(uint32_t *ctr, uint32_t target, uint32_t *status)
+{
+    __shared__ int ok;
+    if (threadIdx.x == 0) {
+        ok = 1;
         const unsigned long long t0 = globaltimer_ns();
         while (true) {
             const uint32_t v = *reinterpret_cast<volatile uint32_t *>(ctr);
@@ -98,6 +110,67 @@ __device__ bool grid_barrier(uint32_t *ctr, uint32_t target, uint32_t *status, b
     }
     __syncthreads();
     return ok != 0;
+}
+
+// Gates of one token from its k selected logits (best first): softmax over
+// the k, or its limit when a selected logit is infinite.
+__device__ __forceinline__ void gates_of(const float *val, int k, float *g)
+{
+    const float m = val[0];
+    if (m == INFINITY) {
+        int cnt = 0;
+        for (int j = 0; j < k; ++j) cnt += (val[j] == INFINITY);
+        for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)cnt : 0.0f;
+    } else if (m == -INFINITY) {
+        for (int j = 0; j < k; ++j) g[j] = 1.0f / (float)k;
+    } else {
+        float z = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            g[j] = expf(val[j] - m);
+            z += g[j];
+        }
+        const float rz = 1.0f / z;
+        for (int j = 0; j < k; ++j) g[j] *= rz;
+    }
+}
+
+// Top-k of one token by one thread: a sorted list of the K best (value,
+// index) pairs in registers, one pass over the N logits at stride `stride`.
+template <int K>
+__device__ __forceinline__ void topk_thread(const RouteParams &p, int t, const float *l, int *sh_hist)
+{
+    float val[K];
+    int sel[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        val[j] = -INFINITY;
+        sel[j] = 0x7fffffff;  // ranks after every real candidate
+    }
+    for (int e = 0; e < p.N; ++e) {
+        const float v = l[e];
+        bool b[K];
+#pragma unroll
+        for (int j = 0; j < K; ++j) b[j] = ranks_before(v, e, val[j], sel[j]);
+#pragma unroll
+        for (int j = K - 1; j > 0; --j) {
+            if (b[j]) {
+                val[j] = b[j - 1] ? val[j - 1] : v;
+                sel[j] = b[j - 1] ? sel[j - 1] : e;
+            }
+        }
+        if (b[0]) {
+            val[0] = v;
+            sel[0] = e;
+        }
+    }
+    float g[K];
+    gates_of(val, K, g);
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        p.topk_idx[(size_t)t * K + j] = sel[j];
+        p.gates[(size_t)t * K + j] = g[j];
+        atomicAdd(&sh_hist[sel[j]], 1);
+    }
 }
 
 // Top-k and gates of one token whose N logits are in shared memory (NaN
@@ -140,22 +213,7 @@ __device__ __forceinline__ void topk_token(const RouteParams &p, int t, const fl
     }
     if (lane == 0) {
         float g[kMaxK];
-        const float m = val[0];
-        if (m == INFINITY) {
-            int cnt = 0;
-            for (int j = 0; j < k; ++j) cnt += (val[j] == INFINITY);
-            for (int j = 0; j < k; ++j) g[j] = (val[j] == INFINITY) ? 1.0f / (float)cnt : 0.0f;
-        } else if (m == -INFINITY) {
-            for (int j = 0; j < k; ++j) g[j] = 1.0f / (float)k;
-        } else {
-            float z = 0.0f;
-            for (int j = 0; j < k; ++j) {
-                g[j] = expf(val[j] - m);
-                z += g[j];
-            }
-            const float rz = 1.0f / z;
-            for (int j = 0; j < k; ++j) g[j] *= rz;
-        }
+        gates_of(val, k, g);
         for (int j = 0; j < k; ++j) {
             p.topk_idx[(size_t)t * k + j] = sel[j];
             p.gates[(size_t)t * k + j] = g[j];
@@ -164,13 +222,18 @@ __device__ __forceinline__ void topk_token(const RouteParams &p, int t, const fl
     }
 }
 
-// Top-k, gates and the histogram of the block's token range [t0, t1):
-// batches of tokens are staged in shared memory with coalesced 16-byte loads
-// (one memory latency per batch), then one warp per token selects.
-__device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, float *sh_logits, int batch,
-                           bool &saw_nan)
+// Top-k, gates and the histogram of the block's token range [t0, t1).
+// Batches of tokens are staged in shared memory with coalesced 16-byte loads
+// (one memory latency per batch; NaN becomes -inf and is reported).  Up to
+// kThreadTopkMaxN experts one thread selects for one token (rows padded to
+// N+1 floats so the threads' column reads hit distinct banks); beyond, one
+// warp per token.
+__device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, float *sh_logits, bool &saw_nan)
 {
     const int N = p.N;
+    const bool per_thread = N <= kThreadTopkMaxN;
+    const int ldl = per_thread ? N + 1 : N;
+    const int batch = route_batch_tokens(N);
     for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     for (int b0 = t0; b0 < t1; b0 += batch) {
@@ -180,24 +243,49 @@ __device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, f
         __syncthreads();
         if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0) {
             const float4 *s4 = reinterpret_cast<const float4 *>(src);
-            float4 *d4 = reinterpret_cast<float4 *>(sh_logits);
             for (size_t q = threadIdx.x; q < nval / 4; q += blockDim.x) {
-                float4 v = __ldg(s4 + q);
-                if (v.x != v.x) { saw_nan = true; v.x = -INFINITY; }
-                if (v.y != v.y) { saw_nan = true; v.y = -INFINITY; }
-                if (v.z != v.z) { saw_nan = true; v.z = -INFINITY; }
-                if (v.w != v.w) { saw_nan = true; v.w = -INFINITY; }
-                d4[q] = v;
+                const float4 v = __ldg(s4 + q);
+                const float f[4] = {v.x, v.y, v.z, v.w};
+                const int tok = (int)((4 * q) / N), e0 = (int)((4 * q) % N);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float x = f[i];
+                    if (x != x) {
+                        saw_nan = true;
+                        x = -INFINITY;
+                    }
+                    sh_logits[(size_t)tok * ldl + e0 + i] = x;
+                }
             }
         } else {
             for (size_t q = threadIdx.x; q < nval; q += blockDim.x) {
-                float v = __ldg(src + q);
-                if (v != v) { saw_nan = true; v = -INFINITY; }
-                sh_logits[q] = v;
+                float x = __ldg(src + q);
+                if (x != x) {
+                    saw_nan = true;
+                    x = -INFINITY;
+                }
+                sh_logits[(q / N) * ldl + q % N] = x;
             }
         }
         __syncthreads();
-        for (int q = warp; q < nb; q += nw) topk_token(p, b0 + q, sh_logits + (size_t)q * N, sh_hist);
+        if (per_thread) {
+            const int q = threadIdx.x;
+            if (q < nb) {
+                const float *l = sh_logits + (size_t)q * ldl;
+                switch (p.k) {
+                case 1: topk_thread<1>(p, b0 + q, l, sh_hist); break;
+                case 2: topk_thread<2>(p, b0 + q, l, sh_hist); break;
+                case 3: topk_thread<3>(p, b0 + q, l, sh_hist); break;
+                case 4: topk_thread<4>(p, b0 + q, l, sh_hist); break;
+                case 5: topk_thread<5>(p, b0 + q, l, sh_hist); break;
+                case 6: topk_thread<6>(p, b0 + q, l, sh_hist); break;
+                case 7: topk_thread<7>(p, b0 + q, l, sh_hist); break;
+                default: topk_thread<8>(p, b0 + q, l, sh_hist); break;
+                }
+            }
+        } else {
+            for (int q = warp; q < nb; q += nw) topk_token(p, b0 + q, sh_logits + (size_t)q * ldl, sh_hist);
+        }
     }
     __syncthreads();
 }
@@ -230,49 +318,68 @@ __device__ __forceinline__ void decode_chunk(const uint32_t *__restrict__ packed
     reinterpret_cast<uint4 *>(wb)[q] = make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// Exclusive scan of src[0..n) into dst[0..n) by the whole block; returns the
-// sum.  `scratch` holds blockDim.x ints.  src and dst may alias.
+// Exclusive scan of src[0..n) into dst[0..n) by the whole block (warp
+// shuffles; `scratch` holds 72 ints); returns the sum.  src and dst may alias.
 __device__ int block_exclusive_scan(const int *src, int *dst, int n, int *scratch)
 {
     const int per = (n + blockDim.x - 1) / blockDim.x;
     const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
     int s = 0;
     for (int e = lo; e < hi; ++e) s += src[e];
-    scratch[threadIdx.x] = s;
-    __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-        const int v = (int)threadIdx.x >= off ? scratch[threadIdx.x - off] : 0;
-        __syncthreads();
-        scratch[threadIdx.x] += v;
-        __syncthreads();
+    int incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
     }
-    int run = scratch[threadIdx.x] - s;
-    const int totalsum = scratch[blockDim.x - 1];
+    if (lane == 31) scratch[warp] = incl;
     __syncthreads();
+    if (warp == 0) {
+        const int w = lane < nw ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += o;
+        }
+        if (lane < nw) scratch[32 + lane] = wi - w;  // exclusive prefix of the warp totals
+        if (lane == nw - 1) scratch[64] = wi;         // block total
+    }
+    __syncthreads();
+    int run = scratch[32 + warp] + incl - s;
+    const int total = scratch[64];
     for (int e = lo; e < hi; ++e) {
         const int v = src[e];
         dst[e] = run;
         run += v;
     }
     __syncthreads();
-    return totalsum;
+    return total;
 }
 
 __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
 {
-    extern __shared__ int sh[];  // phase A: hist[N]; phase C: off[N+1], tstart[N+1], cnt[N], scratch[256]
+    extern __shared__ int sh[];  // phase A: hist[N] + staged logits; phase C: off, tstart, cnt, scratch
     const int N = p.N, k = p.k;
-    const int nchunk = gridDim.x;  // one histogram row per block
+    const int nblk = gridDim.x;  // one histogram row per block
 
-    // ---- phase A: top-k over this block's token range, plus the prep work
-    float *sh_logits = reinterpret_cast<float *>(sh + N);
-    const int batch = route_batch_tokens(N);
+    BFMOE_TRACE(0, threadIdx.x == 0, 0);
+    // ---- phase A: top-k over this block's token range
+    float *sh_logits = reinterpret_cast<float *>(sh + ((N + 3) & ~3));
     bool saw_nan = false;
-    const int tpb = (p.T + gridDim.x - 1) / gridDim.x;  // tokens per block
+    const int tpb = (p.T + nblk - 1) / nblk;  // tokens per block
     const int t0 = min(p.T, (int)blockIdx.x * tpb), t1 = min(p.T, t0 + tpb);
-    topk_range(p, t0, t1, sh, sh_logits, batch, saw_nan);
+    topk_range(p, t0, t1, sh, sh_logits, saw_nan);
     for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)blockIdx.x * N + e] = sh[e];
     if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
+    BFMOE_TRACE(0, threadIdx.x == 0, 1);
+    const bool arrive = (int)blockIdx.x != p.skip_arrive_block;  // test hook: one block never arrives
+    if (arrive) grid_arrive(p.sync);
+
+    // ---- while the other blocks finish their top-k: cos/sin tables and the
+    // decoded base (forward only)
     const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t gthreads = (size_t)gridDim.x * blockDim.x;
     if (p.coef_t) {
@@ -280,7 +387,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             const bool second = i >= (size_t)p.ncoef;
             const size_t j = second ? i - p.ncoef : i;
             float s, c;
-            sincosf(second ? p.phi[j] : p.theta[j], &s, &c);
+            __sincosf(second ? p.phi[j] : p.theta[j], &s, &c);
             (second ? p.coef_p : p.coef_t)[j] = make_float2(c, s);
         }
     }
@@ -290,49 +397,62 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         const size_t nq = (size_t)p.d * p.d / 8;
         for (size_t q = gtid; q < nq; q += gthreads) decode_chunk(p.packed, p.d, p.wdec, q);
     }
-    if ((int)blockIdx.x == p.skip_arrive_block) return;  // test hook: never arrive
-    if (!grid_barrier(p.sync, gridDim.x, p.status, true)) return;
+    BFMOE_TRACE(0, threadIdx.x == 0, 2);
+    if (!arrive) return;
+    if (!grid_wait(p.sync, nblk, p.status)) return;
+    BFMOE_TRACE(0, threadIdx.x == 0, 3);
 
-    // ---- phase B: per-expert prefix over chunks
+    // ---- phase B: per-expert exclusive prefix over the blocks
     {
         const int warp = (int)(gtid >> 5), lane = threadIdx.x & 31;
         const int nwarps = (int)(gthreads >> 5);
+        constexpr int kPerLane = kMaxRouteBlocks / 32;
         for (int e = warp; e < N; e += nwarps) {
+            int v[kPerLane];
+#pragma unroll
+            for (int q = 0; q < kPerLane; ++q) {
+                const int c = q * 32 + lane;
+                v[q] = c < nblk ? p.hist[(size_t)c * N + e] : 0;
+            }
             int running = 0;
-            for (int c0 = 0; c0 < nchunk; c0 += 32) {
-                const int c = c0 + lane;
-                const int v = c < nchunk ? p.hist[(size_t)c * N + e] : 0;
-                int incl = v;
+#pragma unroll
+            for (int q = 0; q < kPerLane; ++q) {
+                if (q * 32 >= nblk) break;
+                int incl = v[q];
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const int o = __shfl_up_sync(0xffffffffu, incl, off);
                     if (lane >= off) incl += o;
                 }
-                if (c < nchunk) p.hist[(size_t)c * N + e] = running + incl - v;
+                const int c = q * 32 + lane;
+                if (c < nblk) p.hist[(size_t)c * N + e] = running + incl - v[q];
                 running += __shfl_sync(0xffffffffu, incl, 31);
             }
             if (lane == 0) p.total[e] = running;
         }
     }
-    if (!grid_barrier(p.sync, 2 * gridDim.x, p.status, true)) return;
+    grid_arrive(p.sync);
+    if (!grid_wait(p.sync, 2 * nblk, p.status)) return;
+    BFMOE_TRACE(0, threadIdx.x == 0, 4);
 
     // ---- phase C: bucket offsets, tile list, ranks and scatter
-    int *off = sh;                // [N+1]
-    int *tstart = off + N + 1;    // [N+1]
-    int *cnt = tstart + N + 1;    // [N]
-    int *scratch = cnt + N;       // [blockDim.x]
+    int *off = sh;              // [N+1]
+    int *tstart = off + N + 1;  // [N+1]
+    int *cnt = tstart + N + 1;  // [N]
+    int *scratch = cnt + N;     // [72]
     for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        off[e] = p.total[e];
-        if (p.in_tiles) tstart[e] = (off[e] + p.tile_rows - 1) / p.tile_rows;
+        const int tot = p.total[e];
+        off[e] = tot;
+        tstart[e] = p.tile_rows > 0 ? (tot + p.tile_rows - 1) / p.tile_rows : 0;
     }
     __syncthreads();
     const int rsum = block_exclusive_scan(off, off, N, scratch);
-    int ntiles = 0;
-    if (p.in_tiles) ntiles = block_exclusive_scan(tstart, tstart, N, scratch);
+    const int ntiles = p.in_tiles ? block_exclusive_scan(tstart, tstart, N, scratch) : 0;
     if (threadIdx.x == 0) {
         off[N] = rsum;
         tstart[N] = ntiles;
     }
+    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)blockIdx.x * N + e];
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= N; e += blockDim.x) p.offsets[e] = off[e];
@@ -346,11 +466,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
                 p.in_tiles[q] = make_int4(e, off[e] + r, min(p.tile_rows, n_e - r), 0);
         }
     }
-    const int lane = threadIdx.x & 31;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)blockIdx.x * N + e];
-    __syncthreads();
     if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const unsigned lt = (1u << lane) - 1u;
         const int i0 = t0 * k, i1 = t1 * k;
         for (int c0 = i0; c0 < i1; c0 += 32) {
             const int i = c0 + lane;
@@ -367,13 +485,15 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             }
         }
     }
+    BFMOE_TRACE(0, threadIdx.x == 0, 5);
     pdl_trigger();
 }
 
 __host__ inline size_t route_smem_bytes(int N)
 {
-    const size_t a = (size_t)N * 4 + (size_t)route_batch_tokens(N) * N * 4;  // phase A
-    const size_t c = (size_t)(3 * N + 2 + kRouteThreads) * 4;              // phase C
+    const size_t ldl = N <= kThreadTopkMaxN ? N + 1 : N;
+    const size_t a = (size_t)((N + 3) & ~3) * 4 + (size_t)route_batch_tokens(N) * ldl * 4;  // phase A
+    const size_t c = (size_t)(3 * N + 2 + 72) * 4;                                          // phase C
     return a > c ? a : c;
 }
 
