@@ -12,6 +12,7 @@
 
 #include "contract.cuh"
 #include "layer.cuh"
+#include "prep.cuh"
 #include "route.cuh"
 
 using namespace bfmoe;
@@ -178,8 +179,8 @@ struct StageRec {
     bool on = false;
 };
 
-const char *const kStageNames[] = {"route", "expert_in", "contract", "combine"};
-constexpr int kNumStages = 4;
+const char *const kStageNames[] = {"route", "prep", "expert_in", "contract", "combine"};
+constexpr int kNumStages = 5;
 
 void mark(StageRec *r, cudaStream_t st)
 {
@@ -267,19 +268,28 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     rp.total = reinterpret_cast<int32_t *>(ws + l.total);
     rp.sync = status + 1;
     rp.status = status;
-    rp.theta = theta;
-    rp.phi = phi;
-    rp.coef_t = ct;
-    rp.coef_p = cp;
-    rp.ncoef = N * L * (d / 2);
-    rp.packed = reinterpret_cast<const uint32_t *>(packed);
-    rp.wdec = wdec;
-    rp.d = d;
     rp.in_tiles = tiles;
     rp.n_in_tiles = ntiles;
     rp.tile_rows = tile_rows_for(d);
+    rp.d = d;
     bfmoe_status s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
+    mark(rec, st);
+
+    PrepParams pp{};
+    pp.theta = theta;
+    pp.phi = phi;
+    pp.coef_t = ct;
+    pp.coef_p = cp;
+    pp.ncoef = N * L * (d / 2);
+    pp.d = d;
+    pp.L = L;
+    pp.packed = reinterpret_cast<const uint32_t *>(packed);
+    pp.wdec = wdec;
+    pp.status = status;
+    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, 4 * sms));
+    if (launch(k_prep, dim3(prep_grid), dim3(256), 0, st, rec == nullptr, false, pp) != cudaSuccess)
+        return BFMOE_ERR_CUDA;
     mark(rec, st);
 
     ExpertInParams ep{};
@@ -294,6 +304,7 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     ep.n_tiles = ntiles;
     ep.max_tiles = max_in_tiles(T_, d, N, k);
     ep.coef_t = ct;
+
     ep.a_blocks = ablk;
     ep.status = status;
     const bool smc = expert_in_smem_coef(d, L);
@@ -483,7 +494,7 @@ bfmoe_status bfmoe_butterfly_apply(const void *x, bfmoe_dtype dt, int rows, int 
     if (rows == 0) return BFMOE_OK;
     const int L = ilog2(d);
     const int ncoef = N * L * (d / 2);
-    k_coef<<<(ncoef + 255) / 256, 256, 0, st>>>(angles, ncoef, coef);
+    k_engine_table<<<(ncoef + 255) / 256, 256, 0, st>>>(angles, N, d, L, transpose != 0, coef);
     const int RT = tile_rows_for(d);
     const size_t smem = rows_smem_bytes(d, 1);
     const unsigned grid = (unsigned)((rows + RT - 1) / RT);

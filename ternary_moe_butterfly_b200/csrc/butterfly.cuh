@@ -14,8 +14,9 @@
 // a thread loads the 2^g values of one row that the pass's g stages mix (a
 // "subset": indices that differ only in bits s0..s1-1), rotates them in
 // registers, and stores them back.  Threads are laid out rows-fastest, so a
-// warp works on up to 32 rows of the same subset and its cos/sin loads are
-// broadcasts whenever those rows share an expert.
+// warp works on up to 32 rows of the same subset; the cos/sin table is laid
+// out in consumption order, so a warp reads it with 16-byte loads that are
+// broadcasts whenever its rows share an expert.
 #pragma once
 
 #include "common.cuh"
@@ -25,67 +26,125 @@ namespace bfmoe {
 // Pair index of the pair (j, j + 2^s) in stage s: j with bit s deleted.
 __host__ __device__ constexpr int pair_of(int j, int s) { return ((j >> (s + 1)) << s) | (j & ((1 << s) - 1)); }
 
+// The ri-th integer whose bit b is clear.
+__host__ __device__ constexpr int insert_zero_bit(int ri, int b) { return ((ri >> b) << (b + 1)) | (ri & ((1 << b) - 1)); }
+
+// Stage split of a butterfly of L stages (6 <= L <= 12) into passes of at
+// most 5 stages: pass pi covers stages [pi*L/np, (pi+1)*L/np), np = ceil(L/5).
+__host__ __device__ inline int npass_of(int L) { return (L + 4) / 5; }
+__host__ __device__ inline void pass_bounds(int L, int pi, int &s0, int &g)
+{
+    const int np = npass_of(L);
+    s0 = pi * L / np;
+    g = (pi + 1) * L / np - s0;
+}
+
+// Engine tables hold each expert's {cos a, +-sin a} in the order the
+// row engine consumes them: passes in execution order, then subsets, then
+// stages in execution order, then the subset's rotations (m ascending among
+// the indices whose local-stage bit is clear).  The sign of B^T is folded
+// in.  engine_entry gives the (stage, pair) of entry r of one expert's table.
+__host__ __device__ inline void engine_entry(int d, int L, bool transpose, int r, int &s, int &p)
+{
+    const int np = npass_of(L), half = d >> 1;
+    int q = 0, off = 0, s0 = 0, g = 1;
+    for (; q < np; ++q) {
+        pass_bounds(L, transpose ? np - 1 - q : q, s0, g);
+        if (r < off + g * half) break;
+        off += g * half;
+    }
+    const int w = r - off;
+    const int per = g << (g - 1);  // entries per subset
+    const int sub = w / per, rr = w % per;
+    const int ql = rr >> (g - 1), ri = rr & ((1 << (g - 1)) - 1);
+    const int ls = transpose ? g - 1 - ql : ql;
+    const int base = ((sub >> s0) << (s0 + g)) | (sub & ((1 << s0) - 1));
+    s = s0 + ls;
+    p = pair_of(base | (insert_zero_bit(ri, ls) << s0), s);
+}
+
+// Delete bit b of x (the inverse of insert_zero_bit).
+__host__ __device__ constexpr int delete_bit(int x, int b) { return ((x >> (b + 1)) << b) | (x & ((1 << b) - 1)); }
+
+// Inverse of engine_entry: the table position of the (stage s, pair p) entry.
+__host__ __device__ inline int engine_pos(int d, int L, bool transpose, int s, int p)
+{
+    const int np = npass_of(L), half = d >> 1;
+    int poff = 0, s0 = 0, g = 1;
+    for (int q = 0; q < np; ++q) {
+        pass_bounds(L, transpose ? np - 1 - q : q, s0, g);
+        if (s >= s0 && s < s0 + g) break;
+        poff += g * half;
+    }
+    const int j = insert_zero_bit(p, s);                // lower element of the pair
+    const int m = (j >> s0) & ((1 << g) - 1);           // position inside the subset
+    const int sub = ((j >> (s0 + g)) << s0) | (j & ((1 << s0) - 1));
+    const int ls = s - s0;
+    const int ql = transpose ? g - 1 - ls : ls;
+    return poff + sub * (g << (g - 1)) + (ql << (g - 1)) + delete_bit(m, ls);
+}
+
 // One "subset" of a row: the 2^G values whose indices differ only in bits
-// S0..S0+G-1, index base | (m << S0).  Deleting bit s is additive over the
-// disjoint bit sets of base and m << S0, so a rotation's table entry is
-// pair_of(base, s) + pair_of(m << S0, s): one runtime term per stage and a
-// compile-time offset per rotation.  cos/sin table: float2 {cos a, sin a},
-// [L][d/2] for one expert.
-template <int G, int S0, bool TRANSPOSE>
-__device__ __forceinline__ void bfly_subset(float *row, int base, const float2 *__restrict__ cf, int half)
+// S0..S0+G-1, index base | (m << S0).  `row` is the shared-window address of
+// the row; `tab` the subset's G * 2^(G-1) table entries, read two at a time.
+template <int G, int S0, bool TRANSPOSE, typename Tab>
+__device__ __forceinline__ void bfly_subset(uint32_t row, int base, Tab tab)
 {
     constexpr int M = 1 << G;
+    constexpr int H = M / 2;  // rotations per stage
     float v[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) v[m] = row[base + (m << S0)];
+    for (int m = 0; m < M; ++m) v[m] = lds_f32(row + 4u * (uint32_t)(base + (m << S0)));
 #pragma unroll
-    for (int q = 0; q < G; ++q) {
-        const int ls = TRANSPOSE ? (G - 1 - q) : q;  // local stage
-        const int s = S0 + ls;
-        const float2 *cs = cf + (size_t)s * half + pair_of(base, s);
+    for (int ql = 0; ql < G; ++ql) {
+        const int ls = TRANSPOSE ? (G - 1 - ql) : ql;
+        float2 c[H];
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-            if (m & (1 << ls)) continue;
-            const float2 c = cs[pair_of(m << S0, s)];
-            const float sn = TRANSPOSE ? -c.y : c.y;
+        for (int i = 0; i < H / 2; ++i) {
+            const float4 w = tab.ld4(ql * H + 2 * i);
+            c[2 * i] = make_float2(w.x, w.y);
+            c[2 * i + 1] = make_float2(w.z, w.w);
+        }
+#pragma unroll
+        for (int ri = 0; ri < H; ++ri) {
+            const int m = insert_zero_bit(ri, ls);
             const float a = v[m], b = v[m + (1 << ls)];
-            v[m] = fmaf(c.x, a, -(sn * b));
-            v[m + (1 << ls)] = fmaf(sn, a, c.x * b);
+            v[m] = fmaf(c[ri].x, a, -(c[ri].y * b));
+            v[m + (1 << ls)] = fmaf(c[ri].y, a, c[ri].x * b);
         }
     }
 #pragma unroll
-    for (int m = 0; m < M; ++m) row[base + (m << S0)] = v[m];
+    for (int m = 0; m < M; ++m) sts_f32(row + 4u * (uint32_t)(base + (m << S0)), v[m]);
 }
 
-// Row r uses the table  coef + sexp[r] * estride  (sexp == nullptr: every
-// row uses `coef`, e.g. one expert's table staged in shared memory).
-template <int G, int S0, bool TRANSPOSE>
-__device__ void bfly_pass(float *tile, int ld, int rows, int d, const int *sexp, const float2 *__restrict__ coef,
-                          size_t estride, int nthreads)
+// One pass over `rows` rows of the tile (shared address `tile`, row stride
+// `ld` floats).  Row r uses the table  tab0 + sexp[r] * estride  (sexp ==
+// nullptr: every row uses tab0); `poff` is the pass's offset in a table.
+template <int G, int S0, bool TRANSPOSE, typename Tab>
+__device__ __forceinline__ void bfly_pass(uint32_t tile, int ld, int rows, int d, const int *sexp, Tab tab0,
+                                          int estride, int poff, int nthreads)
 {
-    const int half = d >> 1;
     const int nsub = d >> G;
     constexpr int S1 = S0 + G;
+    constexpr int PER = G << (G - 1);
     const int items = rows * nsub;
     for (int it = threadIdx.x; it < items; it += nthreads) {
         const int r = it % rows;
         const int sub = it / rows;
         const int base = ((sub >> S0) << S1) | (sub & ((1 << S0) - 1));
-        const float2 *cf = sexp ? coef + (size_t)sexp[r] * estride : coef;
-        bfly_subset<G, S0, TRANSPOSE>(tile + (size_t)r * ld, base, cf, half);
+        const Tab tab = tab0 + ((sexp ? sexp[r] * estride : 0) + poff + sub * PER);
+        bfly_subset<G, S0, TRANSPOSE>(tile + 4u * (uint32_t)(r * ld), base, tab);
     }
 }
 
-// Stage split of a butterfly of L stages into passes of at most 5 stages:
-// pass q covers stages [q*L/np, (q+1)*L/np), np = ceil(L/5).
-template <bool TRANSPOSE>
-__device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, float *tile, int ld, int rows, int d,
-                                                   const int *sexp, const float2 *coef, size_t estride)
+template <bool TRANSPOSE, typename Tab>
+__device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, uint32_t tile, int ld, int rows, int d,
+                                                   const int *sexp, Tab tab0, int estride, int poff)
 {
     const int nt = blockDim.x;
 #define BFLY_CASE(LL, PP, GG, SS)                                                                     \
     if (L == LL && pass == PP) {                                                                      \
-        bfly_pass<GG, SS, TRANSPOSE>(tile, ld, rows, d, sexp, coef, estride, nt);                     \
+        bfly_pass<GG, SS, TRANSPOSE>(tile, ld, rows, d, sexp, tab0, estride, poff, nt);               \
         return;                                                                                       \
     }
     BFLY_CASE(6, 0, 3, 0) BFLY_CASE(6, 1, 3, 3)
@@ -99,26 +158,32 @@ __device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, float *tile,
 }
 
 // Apply B (transpose == false) or B^T (transpose == true) to every row r <
-// rows of the tile; row r uses the table of expert sexp[r] (tables of
-// L*d/2 entries, back to back) or, with sexp == nullptr, the single table
-// `coef`.  6 <= L <= 12.  Must be called by all threads of the block (has
-// __syncthreads).
-__device__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int *sexp, const float2 *coef,
-                          bool transpose)
+// rows of the shared-memory tile `tile`; row r uses the engine table (for
+// that direction) of expert sexp[r] (tables of L*d/2 entries, back to back)
+// or, with sexp == nullptr, the single table tab0.  6 <= L <= 12.  Must be
+// called by all threads of the block (has __syncthreads).
+template <typename Tab>
+__device__ __forceinline__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int *sexp, Tab tab0,
+                                          bool transpose)
 {
-    const size_t estride = (size_t)L * (d >> 1);
-    const int npass = (L + 4) / 5;
-    for (int q = 0; q < npass; ++q) {
-        const int pi = transpose ? (npass - 1 - q) : q;
+    const uint32_t ts = smem_addr(tile);
+    const int estride = L * (d >> 1);
+    const int np = npass_of(L);
+    int poff = 0;
+    for (int q = 0; q < np; ++q) {
+        const int pi = transpose ? (np - 1 - q) : q;
+        int s0, g;
+        pass_bounds(L, pi, s0, g);
         if (transpose)
-            bfly_pass_dispatch<true>(L, pi, tile, ld, rows, d, sexp, coef, estride);
+            bfly_pass_dispatch<true>(L, pi, ts, ld, rows, d, sexp, tab0, estride, poff);
         else
-            bfly_pass_dispatch<false>(L, pi, tile, ld, rows, d, sexp, coef, estride);
+            bfly_pass_dispatch<false>(L, pi, ts, ld, rows, d, sexp, tab0, estride, poff);
+        poff += g * (d >> 1);
         __syncthreads();
     }
 }
 
-// Rows per shared-memory tile: up to 32, at most 16384 floats of data.
-__host__ __device__ constexpr int tile_rows_for(int d) { return (16384 / d) < 32 ? (16384 / d) : 32; }
+// Rows per shared-memory tile: up to 16, at most 16384 floats of data.
+__host__ __device__ constexpr int tile_rows_for(int d) { return (16384 / d) < 16 ? (16384 / d) : 16; }
 
 }  // namespace bfmoe

@@ -226,6 +226,66 @@ __device__ __forceinline__ void tmem_ld4_nowait(uint32_t taddr, float &a, float 
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ------------------------------------------------ explicit shared memory --
+// Typed accesses through 32-bit shared-window addresses, so that the loads and
+// stores are shared-memory instructions whatever the compiler can prove
+// about a pointer's origin.
+__device__ __forceinline__ float lds_f32(uint32_t a)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) { asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory"); }
+__device__ __forceinline__ float2 lds_f32x2(uint32_t a)
+{
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t a)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+
+// A cos/sin table that lives in shared memory (address) or global memory.
+struct SmemTab {
+    uint32_t base;  // shared-window byte address of entry 0
+    __device__ __forceinline__ float2 ld2(int i) const { return lds_f32x2(base + 8u * (uint32_t)i); }
+    __device__ __forceinline__ float4 ld4(int i) const { return lds_f32x4(base + 8u * (uint32_t)i); }  // entries i, i+1
+    __device__ __forceinline__ SmemTab operator+(int i) const { return SmemTab{base + 8u * (uint32_t)i}; }
+};
+struct GmemTab {
+    const float2 *p;
+    __device__ __forceinline__ float2 ld2(int i) const { return __ldg(p + i); }
+    __device__ __forceinline__ float4 ld4(int i) const { return __ldg(reinterpret_cast<const float4 *>(p + i)); }
+    __device__ __forceinline__ GmemTab operator+(int i) const { return GmemTab{p + i}; }
+};
+
+// Copy n elements global -> shared by the threads tid = 0..nthr-1: each
+// thread issues a batch of 8 loads into registers before storing any of
+// them, so the loads overlap (a copy loop that interleaves loads and stores
+// through possibly aliasing pointers would wait out every load).
+template <typename T>
+__device__ __forceinline__ void copy_g2s(const T *__restrict__ src, T *dst, int n, int tid, int nthr)
+{
+    for (int q0 = tid; q0 < n; q0 += 8 * nthr) {
+        T v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + u * nthr;
+            if (q < n) v[u] = __ldcg(src + q);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + u * nthr;
+            if (q < n) dst[q] = v[u];
+        }
+    }
+}
+
 // ------------------------------------------------ programmatic dependent launch --
 
 // Wait until the grids this grid depends on have completed and their memory

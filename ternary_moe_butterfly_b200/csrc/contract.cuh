@@ -34,13 +34,51 @@ namespace bfmoe {
 constexpr int kContractThreads = 320;  // 2 control warps + 8 epilogue warps
 constexpr int kStages = 3;
 
-// log2 of the output slice width: the output-butterfly stages the epilogue
-// applies.
-__host__ __device__ constexpr int slice_stages(int BN) { return BN == 256 ? 8 : (BN == 128 ? 7 : 6); }
 
 // Shared-memory cos/sin tables staged per pair of epilogue warps: two
 // experts x slice_stages(BN) stages x BN/2 pairs.
 __host__ __device__ constexpr int pair_table_floats2(int BN) { return 2 * slice_stages(BN) * (BN / 2); }
+
+// Output tables hold each expert's {cos a, sin a} of phi in the order the
+// epilogue and the combine consume them.  For each BN-column slice nh:
+//   pass 1: 32-column blocks blk, stages 0..4, rotations m (bit s clear)
+//           ascending: 80 entries per block;
+//   pass 2: 8-column groups g, stages 5..SIN-1, columns q = 0..7, rotations
+//           over m (columns 8g + q + 32 m) with the stage's bit clear.
+// Then, for the combine, columns c < BN: stages SIN..L-1, rotations over m
+// (columns c + BN m).  out_entry gives the (stage, pair) of entry r.
+__host__ __device__ inline void out_table_entry(int d, int L, int r, int &s, int &p)
+{
+    const int BN = gemm_bn(d), SIN = slice_stages(BN);
+    const int slice = SIN * (BN / 2), NH = d / BN;
+    if (r < NH * slice) {
+        const int nh = r / slice;
+        int w = r % slice;
+        const int p1 = (BN / 32) * 80;
+        int jj;
+        if (w < p1) {
+            const int blk = w / 80, rr = w % 80;
+            s = rr / 16;
+            jj = blk * 32 + insert_zero_bit(rr % 16, s);
+        } else {
+            w -= p1;
+            const int G2 = SIN - 5, M2h = 1 << (G2 - 1);
+            const int per = G2 * 8 * M2h;
+            const int grp = w / per, rr = w % per;
+            const int ls = rr / (8 * M2h), rem = rr % (8 * M2h);
+            s = 5 + ls;
+            jj = grp * 8 + rem / M2h + 32 * insert_zero_bit(rem % M2h, ls);
+        }
+        p = nh * (BN / 2) + pair_of(jj, s);
+    } else {
+        const int w = r - NH * slice;
+        const int HS = L - SIN, per = HS << (HS - 1);
+        const int c = w / per, rr = w % per;
+        const int ls = rr >> (HS - 1);
+        s = SIN + ls;
+        p = pair_of(c + BN * insert_zero_bit(rr & ((1 << (HS - 1)) - 1), ls), s);
+    }
+}
 
 struct ContractParams {
     const __half *a_blocks;   // [Rp/128][d/64] blocks of 128 x 64
@@ -48,7 +86,7 @@ struct ContractParams {
     float *slot;              // [R][d] fp32, token order (row i = t*k + j)
     const int32_t *perm;      // bucket position -> i
     const int32_t *topk_idx;  // i -> expert
-    const float2 *coef_p;     // [N][L][d/2] {cos, sin} of phi
+    const float2 *coef_p;     // [N][L*d/2] output table (see out_table_entry)
     int d, L, N, R, Rp;
     uint32_t *status;
 };
@@ -63,6 +101,25 @@ __device__ __forceinline__ void rot(float &a, float &b, float2 cs)
     const float x = a, y = b;
     a = fmaf(cs.x, x, -(cs.y * y));
     b = fmaf(cs.y, x, cs.x * y);
+}
+
+// Inverse of out_table_entry: the output-table position of (stage s, pair p).
+__host__ __device__ inline int out_pos(int d, int L, int s, int p)
+{
+    const int BN = gemm_bn(d), SIN = slice_stages(BN);
+    const int slice = SIN * (BN / 2), NH = d / BN, NB = BN / 32;
+    if (s < SIN) {
+        const int nh = p / (BN / 2);
+        const int jj = insert_zero_bit(p % (BN / 2), s);  // column inside the slice
+        if (s < 5) return nh * slice + (jj >> 5) * 80 + s * 16 + delete_bit(jj & 31, s);
+        const int G2 = SIN - 5, M2h = 1 << (G2 - 1), PER2 = G2 * 8 * M2h;
+        const int ls = s - 5, c = jj & 31, m = jj >> 5;
+        return nh * slice + NB * 80 + (c >> 3) * PER2 + (ls * 8 + (c & 7)) * M2h + delete_bit(m, ls);
+    }
+    const int HS = L - SIN, pc = HS << (HS - 1);
+    const int jj = insert_zero_bit(p, s);
+    const int c = jj % BN, m = jj / BN, ls = s - SIN;
+    return NH * slice + c * pc + (ls << (HS - 1)) + delete_bit(m, ls);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
@@ -88,60 +145,73 @@ __device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred)
 
 // Output-butterfly stages 0 .. log2(BN)-1 of one row held in TMEM columns
 // [tbase, tbase + BN) of this warp's lanes, then store to `out` (if
-// non-null).  Two warps share the row's lanes: `part` (0 or 1) selects which
-// half of the 32-column blocks (pass 1) and of the column groups (pass 2)
-// this warp takes; `bar_id` is a 64-thread named barrier for the pair.
-template <int BN>
-__device__ __forceinline__ void epilogue_row(uint32_t tbase, const float2 *__restrict__ cf, int cstride,
-                                             float *__restrict__ out, int part, int bar_id)
+// non-null).  `tab` is the row's expert's slice table in the output-table
+// order (shared or global memory, as the caller's pointer type says).  Two
+// warps share the row's lanes: `part` (0 or 1) selects which half of the
+// 32-column blocks (pass 1) and of the 8-column groups (pass 2) this warp
+// takes; `bar_id` is a 64-thread named barrier for the pair.
+template <int BN, typename Tab>
+__device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, float *__restrict__ out, int part,
+                                             int bar_id)
 {
     constexpr int SIN = slice_stages(BN);
-    constexpr int G2 = SIN - 5;                              // stages at stride >= 32
+    constexpr int G2 = SIN - 5;  // stages at stride >= 32
     constexpr int M2 = 1 << G2;
     constexpr int NB = BN / 32;
+    constexpr int PER2 = G2 * 8 * (M2 / 2);
     // pass 1: stages 0..4 inside each 32-column block
 #pragma unroll 1
     for (int blk = part * (NB / 2); blk < (part + 1) * (NB / 2); ++blk) {
         float v[32];
         tmem_ld32(tbase + (uint32_t)(blk * 32), v);
+        const Tab t4 = tab + blk * 80;
 #pragma unroll
         for (int s = 0; s < 5; ++s) {
-            const float2 *cs = cf + s * cstride + pair_of(blk * 32, s);
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                if (m & (1 << s)) continue;
-                rot(v[m], v[m + (1 << s)], cs[pair_of(m, s)]);
+            for (int i = 0; i < 8; ++i) {
+                const float4 w = t4.ld4(s * 16 + 2 * i);
+                const int m0 = insert_zero_bit(2 * i, s), m1 = insert_zero_bit(2 * i + 1, s);
+                rot(v[m0], v[m0 + (1 << s)], make_float2(w.x, w.y));
+                rot(v[m1], v[m1 + (1 << s)], make_float2(w.z, w.w));
             }
         }
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
     }
     tmem_st_wait();
+    BFMOE_TRACE(2, threadIdx.x == 64, 9);
     named_bar_sync(bar_id, 64);
-    // pass 2: stages 5..SIN-1 on columns c + 32 m
+    BFMOE_TRACE(2, threadIdx.x == 64, 10);
+    // pass 2: stages 5..SIN-1 on columns c0 + q + 32 m, 8-column groups
 #pragma unroll 1
-    for (int c0 = part * 16; c0 < part * 16 + 16; c0 += 4) {
-        float v[4][M2];
+    for (int grp = part * 2; grp < part * 2 + 2; ++grp) {
+        const int c0 = grp * 8;
+        float v[8][M2];
 #pragma unroll
-        for (int m = 0; m < M2; ++m)
+        for (int m = 0; m < M2; ++m) {
             tmem_ld4_nowait(tbase + (uint32_t)(c0 + 32 * m), v[0][m], v[1][m], v[2][m], v[3][m]);
+            tmem_ld4_nowait(tbase + (uint32_t)(c0 + 4 + 32 * m), v[4][m], v[5][m], v[6][m], v[7][m]);
+        }
         tmem_ld_wait();
+        const Tab t2 = tab + (NB * 80 + grp * PER2);
 #pragma unroll
         for (int ls = 0; ls < G2; ++ls) {
-            const int s = 5 + ls;
-            const float2 *cs = cf + s * cstride + pair_of(c0, s);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 8; ++q) {
 #pragma unroll
-                for (int m = 0; m < M2; ++m) {
-                    if (m & (1 << ls)) continue;
-                    rot(v[q][m], v[q][m + (1 << ls)], cs[pair_of(q + 32 * m, s)]);
+                for (int ri = 0; ri < M2 / 2; ++ri) {
+                    const int m = insert_zero_bit(ri, ls);
+                    rot(v[q][m], v[q][m + (1 << ls)], t2.ld2((ls * 8 + q) * (M2 / 2) + ri));
                 }
             }
         }
         if (out) {
+            // one full 32-byte sector per lane and instruction
 #pragma unroll
             for (int m = 0; m < M2; ++m)
-                *reinterpret_cast<float4 *>(out + c0 + 32 * m) = make_float4(v[0][m], v[1][m], v[2][m], v[3][m]);
+                asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(out + c0 + 32 * m),
+                             "f"(v[0][m]), "f"(v[1][m]), "f"(v[2][m]), "f"(v[3][m]), "f"(v[4][m]), "f"(v[5][m]),
+                             "f"(v[6][m]), "f"(v[7][m])
+                             : "memory");
         }
     }
 }
@@ -279,17 +349,20 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
                 if (i < 0 || i >= p.R) i = -1;
                 else e = min(max(p.topk_idx[i], 0), p.N - 1);
             }
-            // the rows are in bucket order: stage the tables of the first and
-            // last row's experts for this slice while the MMA runs
+            // the rows are in bucket order: stage the slice tables of the
+            // first and last row's experts while the MMA runs
             const int ea = __shfl_sync(0xffffffffu, e, 0), eb = __shfl_sync(0xffffffffu, e, 31);
             named_bar_sync(bar_id, 64);  // the pair is done with the previous unit's tables
-            for (int q = pt; q < 2 * SIN * (HB / 2); q += 64) {
-                const int t = q / (SIN * (HB / 2)), rem = q % (SIN * (HB / 2));
-                const int sidx = rem / (HB / 2), w = rem % (HB / 2);
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    p.coef_p + ((size_t)(t ? eb : ea) * p.L + sidx) * half + (size_t)nh * HB);
-                reinterpret_cast<float4 *>(ptab + (size_t)(t * SIN + sidx) * HB)[w] = __ldg(src + w);
+            {
+                // the two experts' slice tables: contiguous copies
+                constexpr int SL4 = SIN * HB / 2;  // float4 per slice table
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+                    copy_g2s(reinterpret_cast<const float4 *>(p.coef_p + (size_t)(t ? eb : ea) * p.L * half +
+                                                              (size_t)nh * SIN * HB),
+                             reinterpret_cast<float4 *>(ptab + (size_t)t * SIN * HB), SL4, pt, 64);
             }
+            BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 13);
             bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
             // both warps sharing these lanes take the same branch (they meet
             // at named barriers inside epilogue_row); the barrier also makes
@@ -301,18 +374,19 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             }
             tc_fence_after();
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 6);
-            const float2 *cf;
-            int cstride;
-            if (e == ea || e == eb) {
-                cf = ptab + (e == ea ? 0 : SIN * HB);
-                cstride = HB;
-            } else {  // a third expert inside 32 rows: read its table from global memory
-                cf = p.coef_p + (size_t)e * p.L * half + (size_t)nh * HB;
-                cstride = half;
-            }
+            BFMOE_TRACE(2, threadIdx.x == 192 && li == 0, 11);
             float *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
-            epilogue_row<BN>(tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16), cf, cstride, out, part, bar_id);
+            const uint32_t tb = tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16);
+            if (__all_sync(0xffffffffu, e == ea || e == eb)) {
+                const SmemTab st{smem_addr(ptab + (e == ea ? 0 : SIN * HB))};
+                epilogue_row<BN>(tb, st, out, part, bar_id);
+            } else {  // a third expert inside these 32 rows (a bucket of fewer than 32
+                // rows): every lane reads its own expert's table from global memory
+                epilogue_row<BN>(tb, GmemTab{p.coef_p + (size_t)e * p.L * half + (size_t)nh * SIN * HB}, out, part,
+                                 bar_id);
+            }
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 7);
+            BFMOE_TRACE(2, threadIdx.x == 192 && li == 0, 12);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);

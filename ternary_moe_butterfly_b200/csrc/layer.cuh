@@ -60,14 +60,20 @@ __global__ void k_pack_base(const int8_t *__restrict__ w, int d, uint32_t *__res
     if (!ok) atomicOr(bad, 1u);
 }
 
-__global__ void k_coef(const float *__restrict__ a, int count, float2 *__restrict__ c)
+// Engine table (see engine_entry) of every expert for one direction, from
+// angles [N][L][d/2].
+__global__ void k_engine_table(const float *__restrict__ angles, int N, int d, int L, bool transpose,
+                               float2 *__restrict__ out)
 {
+    const int tab = L * (d / 2);
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < count) {
-        float s, co;
-        sincosf(a[i], &s, &co);
-        c[i] = make_float2(co, s);
-    }
+    if (i >= N * tab) return;
+    const int e = i / tab, r = i % tab;
+    int s, p;
+    engine_entry(d, L, transpose, r, s, p);
+    float sn, cs;
+    sincosf(angles[((size_t)e * L + s) * (d / 2) + p], &sn, &cs);
+    out[i] = make_float2(cs, transpose ? -sn : sn);
 }
 
 // ------------------------------------------------------- tile row I/O --
@@ -128,7 +134,7 @@ struct ExpertInParams {
     const int4 *tiles;       // single-expert row tiles {expert, row0, nrows, -}
     const int32_t *n_tiles;
     int max_tiles;           // capacity of `tiles`
-    const float2 *coef_t;    // [N][L][d/2] {cos, sin} of theta
+    const float2 *coef_t;    // [N][L*d/2] engine table of theta (B^T order)
     __half *a_blocks;        // fp16 operand blocks, rows in bucket order
     uint32_t *status;
 };
@@ -164,11 +170,7 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
         if (r0 < 0 || r0 > p.R - nr) nr = 0;
         if (nr == 0) continue;  // uniform across the block
         const float2 *gtab = p.coef_t + (size_t)e * tab;
-        if (SMEM_COEF) {
-            const float4 *src = reinterpret_cast<const float4 *>(gtab);
-            float4 *dst = reinterpret_cast<float4 *>(sc);
-            for (size_t q = threadIdx.x; q < tab / 2; q += blockDim.x) dst[q] = __ldg(src + q);
-        }
+        BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 5);
         if ((int)threadIdx.x < RT) {
             int t = -1;
             const int r = r0 + (int)threadIdx.x;
@@ -180,44 +182,53 @@ __global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
         }
         __syncthreads();
         // gather: lane = tile row, warp = 16-byte column chunk, so the scalar
-        // shared-memory stores of a warp hit 32 distinct banks; each lane
-        // issues a batch of 8 loads before converting any of them
-        {
-            const int t = lane < nr ? stok[lane] : -1;
-            constexpr int VPC = 16 / sizeof(T);  // values per 16-byte chunk
-            const int nchunk = d / VPC;
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(t >= 0 ? t : 0) * d);
-            float *dst = tile + (size_t)lane * ld;
-            for (int c0 = warp; c0 < nchunk; c0 += 8 * nw) {
-                uint4 u[8];
+        // shared-memory stores of a warp hit 32 distinct banks; the first
+        // batch of loads is issued before the expert's table is built, so
+        // the two overlap
+        BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 6);
+        const int t_lane = lane < nr ? stok[lane] : -1;
+        constexpr int VPC = 16 / sizeof(T);  // values per 16-byte chunk
+        const int nchunk = d / VPC;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(t_lane >= 0 ? t_lane : 0) * d);
+        float *dst = tile + (size_t)lane * ld;
+        for (int c0 = warp; c0 < nchunk; c0 += 8 * nw) {
+            uint4 u[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int c = c0 + q * nw;
+                u[q] = (t_lane >= 0 && c < nchunk) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            }
+            if (SMEM_COEF && c0 == warp) {
+                // stage the expert's table (contiguous) while the row loads fly
+                copy_g2s(reinterpret_cast<const float4 *>(gtab), reinterpret_cast<float4 *>(sc), (int)tab / 2,
+                         threadIdx.x, blockDim.x);
+                BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 7);
+            }
+            if (lane < nr) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int c = c0 + q * nw;
-                    u[q] = (t >= 0 && c < nchunk) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                }
-                if (lane < nr) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int c = c0 + q * nw;
-                        if (c >= nchunk) break;
-                        float f[8];
-                        if (VPC == 8) {
-                            unpack_bf16x8(u[q], f);
-                        } else {
-                            f[0] = __uint_as_float(u[q].x);
-                            f[1] = __uint_as_float(u[q].y);
-                            f[2] = __uint_as_float(u[q].z);
-                            f[3] = __uint_as_float(u[q].w);
-                        }
-#pragma unroll
-                        for (int i = 0; i < VPC; ++i) dst[c * VPC + i] = f[i];
+                    if (c >= nchunk) break;
+                    float f[8];
+                    if (VPC == 8) {
+                        unpack_bf16x8(u[q], f);
+                    } else {
+                        f[0] = __uint_as_float(u[q].x);
+                        f[1] = __uint_as_float(u[q].y);
+                        f[2] = __uint_as_float(u[q].z);
+                        f[3] = __uint_as_float(u[q].w);
                     }
+#pragma unroll
+                    for (int i = 0; i < VPC; ++i) dst[c * VPC + i] = f[i];
                 }
             }
         }
         __syncthreads();
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 3);
-        bfly_tile(tile, ld, nr, d, L, nullptr, SMEM_COEF ? sc : gtab, /*transpose=*/true);
+        if (SMEM_COEF)
+            bfly_tile(tile, ld, nr, d, L, nullptr, SmemTab{smem_addr(sc)}, /*transpose=*/true);
+        else
+            bfly_tile(tile, ld, nr, d, L, nullptr, GmemTab{gtab}, /*transpose=*/true);
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 4);
         bool overflow = false;
         const int nch = nr * (d / 8);
@@ -255,7 +266,7 @@ struct CombineParams {
     int s_lo;                 // first output stage left to apply (log2 of the GEMM's N tile)
     const int32_t *topk_idx;
     const float *gates;
-    const float2 *coef_p;     // [N][L][d/2]
+    const float2 *coef_p;     // [N][L*d/2] output table (see out_table_entry)
     const uint32_t *packed;   // alpha in word 2
     void *y;
 };
@@ -289,27 +300,19 @@ __global__ void __launch_bounds__(256) k_combine_high(CombineParams p)
             const float g = p.gates[i];
             const float *row = p.slot + (size_t)i * d;
             float v[G];
-            float2 cs[HS][G / 2];
-            const float2 *cf = p.coef_p + (size_t)e * p.L * half;
+            float2 cs[HS * (G / 2)];
+            // this column's entries of the output table: stages s_lo.., rotations
+            const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)p.s_lo * half + (size_t)c * (HS * (G / 2));
 #pragma unroll
             for (int m = 0; m < G; ++m) v[m] = row[c + 256 * m];
 #pragma unroll
-            for (int ls = 0; ls < HS; ++ls) {
-                const int s = p.s_lo + ls;
-                int q = 0;
-#pragma unroll
-                for (int m = 0; m < G; ++m) {
-                    if (m & (1 << ls)) continue;
-                    cs[ls][q++] = __ldg(cf + (size_t)s * half + pair_of(c + 256 * m, s));
-                }
-            }
+            for (int q = 0; q < HS * (G / 2); ++q) cs[q] = __ldg(cf + q);
 #pragma unroll
             for (int ls = 0; ls < HS; ++ls) {
-                int q = 0;
 #pragma unroll
-                for (int m = 0; m < G; ++m) {
-                    if (m & (1 << ls)) continue;
-                    const float2 w = cs[ls][q++];
+                for (int ri = 0; ri < G / 2; ++ri) {
+                    const int m = insert_zero_bit(ri, ls);
+                    const float2 w = cs[ls * (G / 2) + ri];
                     const float a = v[m], b = v[m + (1 << ls)];
                     v[m] = fmaf(w.x, a, -(w.y * b));
                     v[m + (1 << ls)] = fmaf(w.y, a, w.x * b);
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(256) k_bfly_apply(const T *__restrict__ x, int
             for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
     }
     __syncthreads();
-    bfly_tile(tile, ld, RT, d, L, sexp, coef, transpose != 0);
+    bfly_tile(tile, ld, RT, d, L, sexp, GmemTab{coef}, transpose != 0);
     const int nch = nr * (d / 8);
     for (int q = threadIdx.x; q < nch; q += blockDim.x) {
         const int rq = q / (d / 8), c8 = q % (d / 8);

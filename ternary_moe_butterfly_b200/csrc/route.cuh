@@ -7,30 +7,38 @@
 // the k selected logits.  Bucketing is a stable counting sort of the rows
 // i = t*k + j by expert, so each bucket lists its rows in token order.
 //
-// Phases, separated by two bounded grid barriers (all blocks are
+// Phases, separated by one or two bounded grid barriers (all blocks are
 // co-resident: the kernel is launched cooperatively):
 //   A  each block takes a contiguous token range; batches of its tokens'
 //      logits are staged in shared memory and one thread (one warp beyond
 //      256 experts) per token selects the top-k; the block counts its rows
-//      per expert (hist[block][e]).  Between arriving at the first barrier
-//      and waiting on it, the blocks turn the butterfly angles into
-//      {cos, sin} tables and decode the packed ternary base into the
-//      tensor-core operand layout (forward only).
-//   B  one warp per expert scans hist[.][e] over the blocks (exclusive
-//      prefix per block, total per expert).
+//      per expert (hist[block][e]).
+//   B  up to 512 experts, every block reads the (expert-major) histogram
+//      and forms the expert totals and its own prefix over the blocks before
+//      it; beyond, one warp per expert scans the column over the blocks and a
+//      second grid barrier publishes the prefixes.
 //   C  every block scans the expert totals into bucket offsets, then ranks
 //      the rows of its tokens inside their buckets (warp match + popcount)
 //      and scatters perm / row_pos; the blocks also write the list of
 //      single-expert row tiles that the input-butterfly kernel walks.
 #pragma once
 
+#include "butterfly.cuh"
 #include "common.cuh"
 
 namespace bfmoe {
 
+__host__ __device__ inline void out_table_entry(int d, int L, int r, int &s, int &p);
+__host__ __device__ inline int out_pos(int d, int L, int s, int p);
+// log2 of the contraction's output slice width BN: the output-butterfly
+// stages its epilogue applies (the rest go to the combine).
+__host__ __device__ constexpr int slice_stages(int BN) { return BN == 256 ? 8 : (BN == 128 ? 7 : 6); }
+
 constexpr int kRouteThreads = 256;
 constexpr int kMaxK = 8;
 constexpr int kMaxRouteBlocks = 512;  // capacity of the per-block histogram
+constexpr int kOneBarrierMaxN = 512;  // up to this many experts the routing needs one grid barrier
+constexpr int kHistStageInts = 8192;  // histogram ints staged per chunk (32 KB)
 constexpr uint32_t kPackMagic = 0x32574642u;  // "BFW2"
 
 __host__ __device__ constexpr int gemm_bn(int d) { return d < 256 ? d : 256; }
@@ -49,12 +57,6 @@ struct RouteParams {
     uint32_t *sync;      // grid barrier counter, zero at launch
     uint32_t *status;
     int skip_arrive_block;  // test hook: this block never reaches barrier 1 (-1: none)
-    // forward only: prep done while routing
-    const float *theta, *phi;
-    float2 *coef_t, *coef_p;
-    int ncoef;
-    const uint32_t *packed;
-    __half *wdec;
     int d;
     // forward only: single-expert row tiles for the input butterfly
     int4 *in_tiles;
@@ -243,28 +245,39 @@ __device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, f
         __syncthreads();
         if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0) {
             const float4 *s4 = reinterpret_cast<const float4 *>(src);
-            for (size_t q = threadIdx.x; q < nval / 4; q += blockDim.x) {
-                const float4 v = __ldg(s4 + q);
-                const float f[4] = {v.x, v.y, v.z, v.w};
-                const int tok = (int)((4 * q) / N), e0 = (int)((4 * q) % N);
+            const int n4 = (int)(nval / 4);
+            for (int q0 = threadIdx.x; q0 < n4; q0 += 8 * blockDim.x) {
+                float4 v[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float x = f[i];
-                    if (x != x) {
-                        saw_nan = true;
-                        x = -INFINITY;
+                for (int u = 0; u < 8; ++u) {
+                    const int q = q0 + u * blockDim.x;
+                    if (q < n4) v[u] = __ldg(s4 + q);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int q = q0 + u * blockDim.x;
+                    if (q >= n4) break;
+                    const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    const int tok = (4 * q) / N, e0 = (4 * q) % N;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float xv = f[i];
+                        if (xv != xv) {
+                            saw_nan = true;
+                            xv = -INFINITY;
+                        }
+                        sh_logits[(size_t)tok * ldl + e0 + i] = xv;
                     }
-                    sh_logits[(size_t)tok * ldl + e0 + i] = x;
                 }
             }
         } else {
             for (size_t q = threadIdx.x; q < nval; q += blockDim.x) {
-                float x = __ldg(src + q);
-                if (x != x) {
+                float xv = __ldg(src + q);
+                if (xv != xv) {
                     saw_nan = true;
-                    x = -INFINITY;
+                    xv = -INFINITY;
                 }
-                sh_logits[(q / N) * ldl + q % N] = x;
+                sh_logits[(q / N) * ldl + q % N] = xv;
             }
         }
         __syncthreads();
@@ -366,44 +379,61 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     const int nblk = gridDim.x;  // one histogram row per block
 
     BFMOE_TRACE(0, threadIdx.x == 0, 0);
+    pdl_trigger();  // the prep kernel may start now and run beside the routing
     // ---- phase A: top-k over this block's token range
     float *sh_logits = reinterpret_cast<float *>(sh + ((N + 3) & ~3));
     bool saw_nan = false;
     const int tpb = (p.T + nblk - 1) / nblk;  // tokens per block
     const int t0 = min(p.T, (int)blockIdx.x * tpb), t1 = min(p.T, t0 + tpb);
     topk_range(p, t0, t1, sh, sh_logits, saw_nan);
-    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)blockIdx.x * N + e] = sh[e];
+    const bool one_barrier = N <= kOneBarrierMaxN;  // one grid barrier
+    const int np4 = (N + 3) & ~3;                    // histogram row stride, 16-byte multiple
+    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)blockIdx.x * (one_barrier ? np4 : N) + e] = sh[e];
     if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     BFMOE_TRACE(0, threadIdx.x == 0, 1);
     const bool arrive = (int)blockIdx.x != p.skip_arrive_block;  // test hook: one block never arrives
     if (arrive) grid_arrive(p.sync);
 
-    // ---- while the other blocks finish their top-k: cos/sin tables and the
-    // decoded base (forward only)
     const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t gthreads = (size_t)gridDim.x * blockDim.x;
-    if (p.coef_t) {
-        for (size_t i = gtid; i < (size_t)2 * p.ncoef; i += gthreads) {
-            const bool second = i >= (size_t)p.ncoef;
-            const size_t j = second ? i - p.ncoef : i;
-            float s, c;
-            __sincosf(second ? p.phi[j] : p.theta[j], &s, &c);
-            (second ? p.coef_p : p.coef_t)[j] = make_float2(c, s);
-        }
-    }
-    if (p.wdec) {
-        if (gtid == 0 && (p.packed[0] != kPackMagic || p.packed[1] != (uint32_t)p.d))
-            set_status(p.status, BFMOE_ERR_INVALID_ARG);
-        const size_t nq = (size_t)p.d * p.d / 8;
-        for (size_t q = gtid; q < nq; q += gthreads) decode_chunk(p.packed, p.d, p.wdec, q);
-    }
     BFMOE_TRACE(0, threadIdx.x == 0, 2);
     if (!arrive) return;
     if (!grid_wait(p.sync, nblk, p.status)) return;
     BFMOE_TRACE(0, threadIdx.x == 0, 3);
 
-    // ---- phase B: per-expert exclusive prefix over the blocks
-    {
+    int *off = sh;              // [N+1]
+    int *tstart = off + N + 1;  // [N+1]
+    int *cnt = tstart + N + 1;  // [N]
+    int *scratch = cnt + N;     // [72]
+    if (one_barrier) {
+        // ---- every block: expert totals and its own prefix over the blocks
+        // before it, from the expert-major histogram, staged in shared memory
+        // in chunks of experts with coalesced 16-byte loads
+        int *stage = sh + ((3 * N + 82 + 3) & ~3);  // [rb * np4], 16-byte aligned
+        const int rb = max(1, kHistStageInts / np4);  // histogram rows per chunk
+        for (int e = threadIdx.x; e < N; e += blockDim.x) {
+            off[e] = 0;
+            cnt[e] = 0;
+        }
+        for (int b0 = 0; b0 < nblk; b0 += rb) {
+            const int nb = min(rb, nblk - b0);
+            copy_g2s(reinterpret_cast<const int4 *>(p.hist + (size_t)b0 * np4), reinterpret_cast<int4 *>(stage),
+                     nb * np4 / 4, threadIdx.x, blockDim.x);
+            __syncthreads();
+            for (int e = threadIdx.x; e < N; e += blockDim.x) {
+                int tot = 0, pre = 0;
+                for (int b = 0; b < nb; ++b) {
+                    const int v = stage[b * np4 + e];
+                    tot += v;
+                    pre += (b0 + b < (int)blockIdx.x) ? v : 0;
+                }
+                off[e] += tot;
+                cnt[e] += pre;  // becomes the block's bucket base below
+            }
+            __syncthreads();
+        }
+    } else {
+        // ---- phase B: one warp per expert, exclusive prefix over the blocks
         const int warp = (int)(gtid >> 5), lane = threadIdx.x & 31;
         const int nwarps = (int)(gthreads >> 5);
         constexpr int kPerLane = kMaxRouteBlocks / 32;
@@ -420,9 +450,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
                 if (q * 32 >= nblk) break;
                 int incl = v[q];
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += o;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += x;
                 }
                 const int c = q * 32 + lane;
                 if (c < nblk) p.hist[(size_t)c * N + e] = running + incl - v[q];
@@ -430,21 +460,19 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             }
             if (lane == 0) p.total[e] = running;
         }
+        grid_arrive(p.sync);
+        if (!grid_wait(p.sync, 2 * nblk, p.status)) return;
+        for (int e = threadIdx.x; e < N; e += blockDim.x) {
+            off[e] = p.total[e];
+            cnt[e] = p.hist[(size_t)blockIdx.x * N + e];
+        }
+        __syncthreads();
     }
-    grid_arrive(p.sync);
-    if (!grid_wait(p.sync, 2 * nblk, p.status)) return;
     BFMOE_TRACE(0, threadIdx.x == 0, 4);
 
     // ---- phase C: bucket offsets, tile list, ranks and scatter
-    int *off = sh;              // [N+1]
-    int *tstart = off + N + 1;  // [N+1]
-    int *cnt = tstart + N + 1;  // [N]
-    int *scratch = cnt + N;     // [72]
-    for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        const int tot = p.total[e];
-        off[e] = tot;
-        tstart[e] = p.tile_rows > 0 ? (tot + p.tile_rows - 1) / p.tile_rows : 0;
-    }
+    for (int e = threadIdx.x; e < N; e += blockDim.x)
+        tstart[e] = p.tile_rows > 0 ? (off[e] + p.tile_rows - 1) / p.tile_rows : 0;
     __syncthreads();
     const int rsum = block_exclusive_scan(off, off, N, scratch);
     const int ntiles = p.in_tiles ? block_exclusive_scan(tstart, tstart, N, scratch) : 0;
@@ -452,7 +480,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         off[N] = rsum;
         tstart[N] = ntiles;
     }
-    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = off[e] + p.hist[(size_t)blockIdx.x * N + e];
+    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] += off[e];
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= N; e += blockDim.x) p.offsets[e] = off[e];
@@ -486,14 +514,13 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         }
     }
     BFMOE_TRACE(0, threadIdx.x == 0, 5);
-    pdl_trigger();
 }
 
 __host__ inline size_t route_smem_bytes(int N)
 {
     const size_t ldl = N <= kThreadTopkMaxN ? N + 1 : N;
     const size_t a = (size_t)((N + 3) & ~3) * 4 + (size_t)route_batch_tokens(N) * ldl * 4;  // phase A
-    const size_t c = (size_t)(3 * N + 2 + 72) * 4;                                          // phase C
+    const size_t c = (size_t)(((3 * N + 82 + 3) & ~3) + kHistStageInts) * 4;               // phase B/C
     return a > c ? a : c;
 }
 
