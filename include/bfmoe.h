@@ -121,6 +121,32 @@ BFMOE_API size_t bfmoe_route_workspace_bytes(int T, int N, int k);
 BFMOE_API bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk_idx, float *gates,
                          int32_t *perm, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* Routing for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a deployment variant of bfmoe_route.
+ *
+ * Some callers have no way to obtain device memory on the path where they
+ * route: a plugin running inside a host framework that owns every
+ * allocation, a real-time loop where allocation is forbidden, or code that
+ * only receives device pointers for its inputs and outputs.  This entry
+ * point takes no workspace: its scratch (status word, grid-barrier counter,
+ * per-block histogram, expert totals) lives in a 1 MiB array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   Arguments and results are those of bfmoe_route (all device memory owned
+ *   by the caller).
+ *   Limits: N <= 510 experts (any T up to the bfmoe_route limit); larger N
+ *   returns BFMOE_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call shares the one array: calls that overlap on the GPU (on
+ *   different streams, or from different threads) race and give undefined
+ *   results; serialise them.  Each call clears the part that must start at
+ *   zero.  Device-side errors (a NaN logit, a timed-out barrier) are not
+ *   reported: a NaN logit ranks as -inf, so the outputs are still a valid
+ *   routing. */
+BFMOE_API bfmoe_status bfmoe_route_static(const float *logits, int T, int N, int k, int32_t *topk_idx, float *gates,
+                                          int32_t *perm, int32_t *offsets, void *stream);
+
 /* ---------------------------------------------------------- butterfly -- */
 
 /* Workspace bytes for bfmoe_butterfly_apply (the cos/sin table). */

@@ -57,6 +57,7 @@ def lib():
             "bfmoe_forward_profile": (I, [P, I, I, I, P, I, I, P, P, P, P, P, Z, P, P, P]),
             "bfmoe_stage_name": (ctypes.c_char_p, [I]),
             "bfmoe_debug_set": (None, [I, I]),
+            "bfmoe_route_static": (I, [P, I, I, I, P, P, P, P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -94,6 +95,11 @@ def bfmoe_route_workspace_bytes(T, N, k):
 
 def bfmoe_route(logits, T, N, k, topk_idx, gates, perm, offsets, ws, ws_bytes, stream):
     return lib().bfmoe_route(logits, T, N, k, topk_idx, gates, perm, offsets, ws, ws_bytes, stream)
+
+
+def bfmoe_route_static(logits, T, N, k, topk_idx, gates, perm, offsets, stream):
+    """bfmoe_route without a workspace (library-held scratch); see include/bfmoe.h."""
+    return lib().bfmoe_route_static(logits, T, N, k, topk_idx, gates, perm, offsets, stream)
 
 
 def bfmoe_butterfly_workspace_bytes(d, N):

@@ -168,6 +168,27 @@ int occupancy(const void *fn, int threads, size_t smem)
 
 bfmoe_status launched() { return cudaGetLastError() == cudaSuccess ? BFMOE_OK : BFMOE_ERR_CUDA; }
 
+// Scratch of bfmoe_route_static, for callers that cannot allocate: one
+// array per device that loads the library, held until the process exits.
+constexpr size_t kStaticScratchBytes = 1u << 20;
+static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
+std::map<int, void *> g_static_scratch;  // device -> device address of g_route_scratch
+
+// The device address of g_route_scratch on the current device (host code
+// cannot use the symbol itself), looked up once per device.
+void *static_scratch()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> g(g_mu);
+    auto it = g_static_scratch.find(dev);
+    if (it != g_static_scratch.end()) return it->second;
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_static_scratch[dev] = ptr;
+    return ptr;
+}
+
 // Process-wide test hook (bfmoe_debug_set): the routing block that skips the
 // first grid barrier, or -1.
 int g_skip_arrive_block = -1;
@@ -439,6 +460,40 @@ bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk
     const RouteLayout l = route_layout(T, N);
     if (ws_bytes < l.total_bytes) return BFMOE_ERR_WORKSPACE;
     uint8_t *w = reinterpret_cast<uint8_t *>(ws);
+    cudaStream_t st = as_stream(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(w + l.status);
+    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
+    RouteParams rp{};
+    rp.logits = logits;
+    rp.T = T;
+    rp.N = N;
+    rp.k = k;
+    rp.topk_idx = topk_idx;
+    rp.gates = gates;
+    rp.perm = perm;
+    rp.offsets = offsets;
+    rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
+    rp.total = reinterpret_cast<int32_t *>(w + l.total);
+    rp.sync = status + 1;
+    rp.status = status;
+    s = launch_route(rp, st);
+    if (s != BFMOE_OK) return s;
+    return launched();
+}
+
+bfmoe_status bfmoe_route_static(const float *logits, int T, int N, int k, int32_t *topk_idx, float *gates,
+                                int32_t *perm, int32_t *offsets, void *stream)
+{
+    bfmoe_status s = check_route_shape(T, N, k);
+    if (s != BFMOE_OK) return s;
+    if (!logits || !topk_idx || !gates || !perm || !offsets) return BFMOE_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(gates, 4) || !aligned(perm, 4) ||
+        !aligned(offsets, 4))
+        return BFMOE_ERR_INVALID_ARG;
+    const RouteLayout l = route_layout(T, N);
+    if (l.total_bytes > kStaticScratchBytes) return BFMOE_ERR_UNSUPPORTED;
+    uint8_t *w = reinterpret_cast<uint8_t *>(static_scratch());
+    if (!w) return BFMOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     uint32_t *status = reinterpret_cast<uint32_t *>(w + l.status);
     if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
