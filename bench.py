@@ -56,6 +56,31 @@ def load_peaks():
     return d
 
 
+def kernel_sources_hash() -> str:
+    import glob
+    import hashlib
+    src = sorted(glob.glob(os.path.join(ROOT, "ternary_moe_butterfly_b200", "csrc", "*")))
+    return hashlib.sha256(b"".join(open(f, "rb").read() for f in src)).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str) -> dict:
+    """DRAM bytes per launch from profiles/traffic.txt, if it was captured on
+    the current kernel sources and this workload (else empty)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return {}
+    meta, vals = {}, {}
+    for line in open(p):
+        parts = line.split()
+        if len(parts) == 3 and parts[0] == "#":
+            meta[parts[1]] = parts[2]
+        elif len(parts) == 2 and not line.startswith("#"):
+            vals[parts[0]] = int(parts[1])
+    if meta.get("source_hash") != kernel_sources_hash() or meta.get("workload") != workload:
+        return {}
+    return vals
+
+
 def layer_model(w: wl.Workload):
     d, N, k, T, L = w.d, w.N, w.k, w.T, w.L
     xb = 2 if w.dtype == "bf16" else 4
@@ -352,7 +377,8 @@ def run_ours(args, w):
             achieved = amount / sec / 1e9
             peak = peaks["hbm_gbs"]
         roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": None, "peak_source": peaks["source"]}
+                "frac": achieved / peak, "traffic": profiled_traffic(w.name).get(dom),
+                "peak_source": peaks["source"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
