@@ -191,9 +191,12 @@ BFMOE_API bfmoe_status bfmoe_forward_ws_layout(int T, int d, int N, int k, bfmoe
  *   theta, phi:  device fp32 [N][L][d/2] (input and output butterflies).
  *   ws:          device workspace of bfmoe_forward_workspace_bytes(T,d,N,k).
  * Precision: rotations and accumulation in fp32; the rotated rows enter the
- * tensor-core contraction as fp16 (W_base's values are exact in fp16); y is
- * rounded to dt.  Device-side errors: NaN logit, fp16 overflow of a rotated
- * row (|x'| > 65504), malformed packed base, timeout. */
+ * tensor-core contraction as fp16 (W_base's values are exact in fp16); each
+ * product row, after the output stages that stay inside one GEMM column tile,
+ * is scaled by alpha * g and held as fp16 until the last stages and the sum
+ * over j; y is rounded to dt.  Device-side errors: NaN logit, fp16 overflow of
+ * a rotated row (|x'| > 65504), non-finite y (fp16 overflow of a scaled
+ * product row), malformed packed base, timeout. */
 BFMOE_API bfmoe_status bfmoe_forward(const void *x, bfmoe_dtype dt, int T, int d, const float *logits, int N, int k,
                            const void *packed_base, const float *theta, const float *phi, void *y, void *ws,
                            size_t ws_bytes, void *stream);

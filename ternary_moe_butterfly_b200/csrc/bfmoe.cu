@@ -108,7 +108,7 @@ FwdLayout fwd_layout(int T, int d, int N, int k)
     l.coef_p = take(ncoef * 8);
     l.wdec = take((size_t)d * d * 2);
     l.a_blocks = take(Rp * d * 2);
-    l.slot = take(R * d * 4);
+    l.slot = take(R * d * 2);
     l.total_bytes = o;
     return l;
 }
@@ -266,7 +266,7 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     float2 *cp = reinterpret_cast<float2 *>(ws + l.coef_p);
     __half *wdec = reinterpret_cast<__half *>(ws + l.wdec);
     __half *ablk = reinterpret_cast<__half *>(ws + l.a_blocks);
-    float *slot = reinterpret_cast<float *>(ws + l.slot);
+    __half *slot = reinterpret_cast<__half *>(ws + l.slot);
     int4 *tiles = reinterpret_cast<int4 *>(ws + l.tiles);
     int32_t *ntiles = reinterpret_cast<int32_t *>(ws + l.ntiles);
     const int sms = device_sms();
@@ -332,9 +332,10 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     const size_t in_smem = expert_in_smem_bytes(d, L, smc);
     auto kin = smc ? k_expert_in<T, true> : k_expert_in<T, false>;
     if (!ensure_smem((const void *)kin, in_smem)) return BFMOE_ERR_CUDA;
-    const int in_occ = occupancy((const void *)kin, 256, in_smem);
+    const int in_occ = occupancy((const void *)kin, kInThreads, in_smem);
     const int in_grid = std::max(1, std::min(max_in_tiles(T_, d, N, k), std::max(1, in_occ) * sms));
-    if (launch(kin, dim3(in_grid), dim3(256), in_smem, st, true, false, ep) != cudaSuccess) return BFMOE_ERR_CUDA;
+    if (launch(kin, dim3(in_grid), dim3(kInThreads), in_smem, st, true, false, ep) != cudaSuccess)
+        return BFMOE_ERR_CUDA;
     mark(rec, st);
 
     ContractParams cpar{};
@@ -344,6 +345,8 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     cpar.perm = perm;
     cpar.topk_idx = idx;
     cpar.coef_p = cp;
+    cpar.gates = gates;
+    cpar.packed = reinterpret_cast<const uint32_t *>(packed);
     cpar.d = d;
     cpar.L = L;
     cpar.N = N;
@@ -369,22 +372,23 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     cb.N = N;
     cb.s_lo = ilog2(BN);
     cb.topk_idx = idx;
-    cb.gates = gates;
     cb.coef_p = cp;
-    cb.packed = reinterpret_cast<const uint32_t *>(packed);
     cb.y = y;
+    cb.status = status;
     const int HS = L - cb.s_lo;
+    const unsigned cthreads = (unsigned)T_ * (unsigned)(BN / 8);  // BN/8 threads per token
+    const dim3 cgrid2((cthreads + 255) / 256);
     cudaError_t e = cudaSuccess;
     switch (HS) {
-    case 0: {
-        const size_t nthreads = (size_t)T_ * (d / 8);
-        e = launch(k_combine_sum<T>, dim3((unsigned)((nthreads + 255) / 256)), dim3(256), 0, st, true, false, cb);
+    case 0:
+        e = BN == 256 ? launch(k_combine<T, 0, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb)
+            : BN == 128 ? launch(k_combine<T, 0, 128, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb)
+                        : launch(k_combine<T, 0, 64, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb);
         break;
-    }
-    case 1: e = launch(k_combine_high<T, 1, 4>, dim3((T_ + 3) / 4), dim3(256), 0, st, true, false, cb); break;
-    case 2: e = launch(k_combine_high<T, 2, 2>, dim3((T_ + 1) / 2), dim3(256), 0, st, true, false, cb); break;
-    case 3: e = launch(k_combine_high<T, 3, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
-    default: e = launch(k_combine_high<T, 4, 1>, dim3(T_), dim3(256), 0, st, true, false, cb); break;
+    case 1: e = launch(k_combine<T, 1, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
+    case 2: e = launch(k_combine<T, 2, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
+    case 3: e = launch(k_combine<T, 3, 256, 4>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
+    default: e = launch(k_combine<T, 4, 256, 2>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
     }
     if (e != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);

@@ -19,7 +19,8 @@
 //            (two warps per row, each on half of the columns) applies the
 //            output-butterfly stages that stay inside the slice
 //            (stages 0 .. log2 BN - 1) to its own row, with the row's expert
-//            table, and stores the fp32 result to the row's token-order slot.
+//            table, scales by alpha * gate and stores fp16 to the row's
+//            token-order slot (the slot layout below).
 //            Stages 0-4 act inside 32-column blocks (one 32-column TMEM load,
 //            rotate, store back); stages 5.. act on columns 32 apart (4-column
 //            TMEM loads).  The remaining stages, which mix slices, are
@@ -83,7 +84,9 @@ __host__ __device__ inline void out_table_entry(int d, int L, int r, int &s, int
 struct ContractParams {
     const __half *a_blocks;   // [Rp/128][d/64] blocks of 128 x 64
     const __half *w_blocks;   // [d/BN][d/64] blocks of BN x 64
-    float *slot;              // [R][d] fp32, token order (row i = t*k + j)
+    __half *slot;             // [R][d] fp16 alpha*gate*u, token order (row i = t*k + j), slot layout
+    const float *gates;       // [R] gate of row i
+    const uint32_t *packed;   // alpha in word 2
     const int32_t *perm;      // bucket position -> i
     const int32_t *topk_idx;  // i -> expert
     const float2 *coef_p;     // [N][L*d/2] output table (see out_table_entry)
@@ -151,19 +154,17 @@ __device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred)
 // 32-column blocks (pass 1) and of the 8-column groups (pass 2) this warp
 // takes; `bar_id` is a 64-thread named barrier for the pair.
 template <int BN, typename Tab>
-__device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, float *__restrict__ out, int part,
-                                             int bar_id)
+__device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__restrict__ out, float scale,
+                                             int part, int bar_id)
 {
     constexpr int SIN = slice_stages(BN);
     constexpr int G2 = SIN - 5;  // stages at stride >= 32
     constexpr int M2 = 1 << G2;
     constexpr int NB = BN / 32;
     constexpr int PER2 = G2 * 8 * (M2 / 2);
-    // pass 1: stages 0..4 inside each 32-column block
-#pragma unroll 1
-    for (int blk = part * (NB / 2); blk < (part + 1) * (NB / 2); ++blk) {
-        float v[32];
-        tmem_ld32(tbase + (uint32_t)(blk * 32), v);
+    // pass 1: stages 0..4 inside each 32-column block; the next block's TMEM
+    // load is in flight while this one rotates
+    auto pass1_block = [&](int blk, float (&v)[32]) {
         const Tab t4 = tab + blk * 80;
 #pragma unroll
         for (int s = 0; s < 5; ++s) {
@@ -176,6 +177,24 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, float *__r
             }
         }
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
+    };
+    {
+        constexpr int NBH = NB / 2;  // blocks per warp
+        const int b0 = part * NBH;
+        float va[32], vb[32];
+        tmem_ld32_async(tbase + (uint32_t)(b0 * 32), va);
+        tmem_ld_wait_regs(va);
+#pragma unroll
+        for (int i = 0; i < NBH; i += 2) {
+            if (i + 1 < NBH) tmem_ld32_async(tbase + (uint32_t)((b0 + i + 1) * 32), vb);
+            pass1_block(b0 + i, va);
+            if (i + 1 < NBH) {
+                tmem_ld_wait_regs(vb);
+                if (i + 2 < NBH) tmem_ld32_async(tbase + (uint32_t)((b0 + i + 2) * 32), va);
+                pass1_block(b0 + i + 1, vb);
+                if (i + 2 < NBH) tmem_ld_wait_regs(va);
+            }
+        }
     }
     tmem_st_wait();
     BFMOE_TRACE(2, threadIdx.x == 64, 9);
@@ -205,12 +224,22 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, float *__r
             }
         }
         if (out) {
-            // one full 32-byte sector per lane and instruction
+            // alpha * gate, fp16, the group's M2 x 8 values as one contiguous run
+            // (slot row layout [group][m][q], described with CombineParams); 32-byte stores
+            uint32_t h[M2 * 4];
 #pragma unroll
             for (int m = 0; m < M2; ++m)
-                asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(out + c0 + 32 * m),
-                             "f"(v[0][m]), "f"(v[1][m]), "f"(v[2][m]), "f"(v[3][m]), "f"(v[4][m]), "f"(v[5][m]),
-                             "f"(v[6][m]), "f"(v[7][m])
+#pragma unroll
+                for (int q = 0; q < 8; q += 2) {
+                    __half2 hv = __floats2half2_rn(scale * v[q][m], scale * v[q + 1][m]);
+                    h[m * 4 + q / 2] = *reinterpret_cast<uint32_t *>(&hv);
+                }
+            __half *dst = out + grp * (8 * M2);
+#pragma unroll
+            for (int w = 0; w < M2 / 2; ++w)
+                asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 16 * w), "r"(h[8 * w]),
+                             "r"(h[8 * w + 1]), "r"(h[8 * w + 2]), "r"(h[8 * w + 3]), "r"(h[8 * w + 4]),
+                             "r"(h[8 * w + 5]), "r"(h[8 * w + 6]), "r"(h[8 * w + 7])
                              : "memory");
         }
     }
@@ -375,15 +404,16 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             tc_fence_after();
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 6);
             BFMOE_TRACE(2, threadIdx.x == 192 && li == 0, 11);
-            float *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
+            __half *out = i >= 0 ? p.slot + (size_t)i * d + (size_t)nh * BN : nullptr;
+            const float scale = i >= 0 ? __uint_as_float(__ldg(p.packed + 2)) * p.gates[i] : 0.0f;
             const uint32_t tb = tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16);
             if (__all_sync(0xffffffffu, e == ea || e == eb)) {
                 const SmemTab st{smem_addr(ptab + (e == ea ? 0 : SIN * HB))};
-                epilogue_row<BN>(tb, st, out, part, bar_id);
+                epilogue_row<BN>(tb, st, out, scale, part, bar_id);
             } else {  // a third expert inside these 32 rows (a bucket of fewer than 32
                 // rows): every lane reads its own expert's table from global memory
-                epilogue_row<BN>(tb, GmemTab{p.coef_p + (size_t)e * p.L * half + (size_t)nh * SIN * HB}, out, part,
-                                 bar_id);
+                epilogue_row<BN>(tb, GmemTab{p.coef_p + (size_t)e * p.L * half + (size_t)nh * SIN * HB}, out, scale,
+                                 part, bar_id);
             }
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 7);
             BFMOE_TRACE(2, threadIdx.x == 192 && li == 0, 12);

@@ -142,8 +142,10 @@ struct ExpertInParams {
 // Persistent over the tile list: gather the rows of one expert's tile, rotate
 // by B(theta_e)^T (the expert's cos/sin table is staged in shared memory when
 // it fits, so every coefficient load is a broadcast), write fp16 A blocks.
+constexpr int kInThreads = 128;  // four CTAs per SM
+
 template <typename T, bool SMEM_COEF>
-__global__ void __launch_bounds__(256) k_expert_in(ExpertInParams p)
+__global__ void __launch_bounds__(kInThreads, 4) k_expert_in(ExpertInParams p)
 {
     extern __shared__ __align__(16) float smem_f[];
     const int d = p.d, L = p.L;
@@ -260,105 +262,137 @@ __host__ inline bool expert_in_smem_coef(int d, int L) { return (size_t)L * (d /
 
 // ------------------------------------------------------------ combine --
 
+// Slot layout.  The contraction epilogue leaves each routed row i = t*k + j
+// as alpha * g_{t,j} * (output butterfly stages 0 .. SIN-1 applied), fp16,
+// d values.  Inside the row, BN-column slice nh holds its columns
+// nh*BN + 8*grp + q + 32*m (grp < 4, q < 8, m < BN/32) at position
+// nh*BN + (grp * (BN/32) + m) * 8 + q: each epilogue thread's 8 x BN/32 values
+// form one contiguous run, and every run of 8 holds 8 consecutive columns.
 struct CombineParams {
-    const float *slot;        // [T*k][d] fp32, rows in token order (i = t*k + j)
+    const __half *slot;       // [T*k][d] fp16, rows in token order (i = t*k + j), slot layout
     int T, d, L, k, N;
     int s_lo;                 // first output stage left to apply (log2 of the GEMM's N tile)
     const int32_t *topk_idx;
-    const float *gates;
     const float2 *coef_p;     // [N][L*d/2] output table (see out_table_entry)
-    const uint32_t *packed;   // alpha in word 2
     void *y;
+    uint32_t *status;
 };
 
-// HS = L - s_lo > 0 high stages: TPB tokens per block, 256 threads; thread c
-// owns columns c + 256 m (m < 2^HS) of each token, which the stages
-// s_lo..L-1 mix.  All slot and table loads of a token are issued before any
-// arithmetic so that each thread keeps many loads in flight.
-template <typename T, int HS, int TPB>
-__global__ void __launch_bounds__(256) k_combine_high(CombineParams p)
+template <typename T>
+__device__ __forceinline__ void store_cols(T *dst, const float *f, int n);
+template <>
+__device__ __forceinline__ void store_cols<float>(float *dst, const float *f, int n)
 {
-    BFMOE_TRACE(3, threadIdx.x == 0, 0);
-    pdl_wait();
-    pdl_trigger();
-    BFMOE_TRACE(3, threadIdx.x == 0, 1);
-    constexpr int G = 1 << HS;
-    const int c = threadIdx.x;
-    const int d = p.d, half = d >> 1;
-    const float alpha = __uint_as_float(__ldg(p.packed + 2));
-#pragma unroll 1
-    for (int tt = 0; tt < TPB; ++tt) {
-        const int t = blockIdx.x * TPB + tt;
-        if (t >= p.T) return;
-        float acc[G];
-#pragma unroll
-        for (int m = 0; m < G; ++m) acc[m] = 0.0f;
-#pragma unroll 1
-        for (int j = 0; j < p.k; ++j) {
-            const int i = t * p.k + j;
-            const int e = min(max(p.topk_idx[i], 0), p.N - 1);
-            const float g = p.gates[i];
-            const float *row = p.slot + (size_t)i * d;
-            float v[G];
-            float2 cs[HS * (G / 2)];
-            // this column's entries of the output table: stages s_lo.., rotations
-            const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)p.s_lo * half + (size_t)c * (HS * (G / 2));
-#pragma unroll
-            for (int m = 0; m < G; ++m) v[m] = row[c + 256 * m];
-#pragma unroll
-            for (int q = 0; q < HS * (G / 2); ++q) cs[q] = __ldg(cf + q);
-#pragma unroll
-            for (int ls = 0; ls < HS; ++ls) {
-#pragma unroll
-                for (int ri = 0; ri < G / 2; ++ri) {
-                    const int m = insert_zero_bit(ri, ls);
-                    const float2 w = cs[ls * (G / 2) + ri];
-                    const float a = v[m], b = v[m + (1 << ls)];
-                    v[m] = fmaf(w.x, a, -(w.y * b));
-                    v[m + (1 << ls)] = fmaf(w.y, a, w.x * b);
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < G; ++m) acc[m] = fmaf(g, v[m], acc[m]);
+    for (int i = 0; i < n; i += 4) *reinterpret_cast<float4 *>(dst + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+}
+template <>
+__device__ __forceinline__ void store_cols<__nv_bfloat16>(__nv_bfloat16 *dst, const float *f, int n)
+{
+    if (n == 8) {
+        *reinterpret_cast<uint4 *>(dst) = pack_bf16x8(f);
+    } else {
+        for (int i = 0; i < n; i += 2) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(f[i], f[i + 1]);
+            *reinterpret_cast<__nv_bfloat162 *>(dst + i) = h;
         }
-        T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d;
-#pragma unroll
-        for (int m = 0; m < G; ++m) store1(y + c + 256 * m, alpha * acc[m]);
     }
 }
 
-// No stage left (d <= 256): 8 columns per thread.
-template <typename T>
-__global__ void __launch_bounds__(256) k_combine_sum(CombineParams p)
+// n consecutive fp16 values (n = 2, 4 or 8, aligned to 2n bytes) as one load
+template <int n>
+__device__ __forceinline__ void load_halves(const __half *src, float *f)
 {
-    pdl_wait();
-    pdl_trigger();
-    const int d = p.d;
-    const int per_tok = d / 8;
-    const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int t = (int)(q / per_tok), c8 = (int)(q % per_tok);
-    if (t >= p.T) return;
-    float f[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = 0.0f;
-    for (int j = 0; j < p.k; ++j) {
-        const int i = t * p.k + j;
-        const float g = p.gates[i];
-        const float4 *src = reinterpret_cast<const float4 *>(p.slot + (size_t)i * d + c8 * 8);
-        const float4 a = src[0], b = src[1];
-        f[0] = fmaf(g, a.x, f[0]);
-        f[1] = fmaf(g, a.y, f[1]);
-        f[2] = fmaf(g, a.z, f[2]);
-        f[3] = fmaf(g, a.w, f[3]);
-        f[4] = fmaf(g, b.x, f[4]);
-        f[5] = fmaf(g, b.y, f[5]);
-        f[6] = fmaf(g, b.z, f[6]);
-        f[7] = fmaf(g, b.w, f[7]);
+    uint32_t w[n / 2];
+    if constexpr (n == 8) {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(src));
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+    } else if constexpr (n == 4) {
+        const uint2 u = __ldcs(reinterpret_cast<const uint2 *>(src));
+        w[0] = u.x, w[1] = u.y;
+    } else {
+        w[0] = __ldcs(reinterpret_cast<const unsigned int *>(src));
     }
-    const float alpha = __uint_as_float(__ldg(p.packed + 2));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] *= alpha;
-    store8<T>(reinterpret_cast<T *>(p.y) + (size_t)t * d + c8 * 8, f);
+    for (int i = 0; i < n / 2; ++i) {
+        __half2 h;
+        *reinterpret_cast<uint32_t *>(&h) = w[i];
+        const float2 x = __half22float2(h);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+// y_t = sum_j (stages s_lo..L-1 of B(phi_e)) slot_{t,j}: the rows arrive
+// already scaled by alpha * g.  HS = L - s_lo stages mix the NH = 2^HS slices
+// (pairs of slices nh, nh + 2^ls at the same in-slice column).  One thread per
+// (token, 8-column group, m) handles QW of the group's 8 columns per round in
+// all NH slices; the k rows are summed in j order.
+template <typename T, int HS, int BN, int QW>
+__global__ void __launch_bounds__(256) k_combine(CombineParams p)
+{
+    BFMOE_TRACE(3, threadIdx.x == 0, 0);
+    pdl_wait();
+    BFMOE_TRACE(3, threadIdx.x == 0, 1);
+    pdl_trigger();
+    constexpr int NH = 1 << HS;
+    constexpr int M2 = BN / 32;
+    constexpr int TPT = 4 * M2;  // threads per token
+    constexpr int PC = HS > 0 ? (HS << (HS - 1)) : 1;  // table entries per column
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+    const int t = tid / TPT;
+    if (t >= p.T) return;
+    const int g = (tid % TPT) / M2, m = tid % M2;
+    const int d = p.d, half = d >> 1;
+    const int col0 = 8 * g + 32 * m;           // first of the thread's 8 in-slice columns
+    const int pos0 = (g * M2 + m) * 8;         // their slot position inside a slice
+    bool bad = false;
+#pragma unroll 1
+    for (int q0 = 0; q0 < 8; q0 += QW) {
+        float acc[NH][QW];
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int q = 0; q < QW; ++q) acc[h][q] = 0.0f;
+#pragma unroll 1
+        for (int j = 0; j < p.k; ++j) {
+            const int i = t * p.k + j;
+            const __half *row = p.slot + (size_t)i * d + pos0 + q0;
+            float v[NH][QW];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) load_halves<QW>(row + h * BN, v[h]);
+            if (HS > 0) {
+                const int e = min(max(p.topk_idx[i], 0), p.N - 1);
+                // combine part of the output table: [column][ls][pair over slices]
+                const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)p.s_lo * half;
+#pragma unroll
+                for (int q = 0; q < QW; ++q) {
+                    const float2 *cq = cf + (size_t)(col0 + q0 + q) * PC;
+#pragma unroll
+                    for (int ls = 0; ls < HS; ++ls)
+#pragma unroll
+                        for (int ri = 0; ri < NH / 2; ++ri) {
+                            const int h = insert_zero_bit(ri, ls);
+                            const float2 w = __ldg(cq + (ls << (HS > 0 ? HS - 1 : 0)) + ri);
+                            const float a = v[h][q], b = v[h + (1 << ls)][q];
+                            v[h][q] = fmaf(w.x, a, -(w.y * b));
+                            v[h + (1 << ls)][q] = fmaf(w.y, a, w.x * b);
+                        }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+#pragma unroll
+                for (int q = 0; q < QW; ++q) acc[h][q] += v[h][q];
+        }
+        T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d + col0 + q0;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+#pragma unroll
+            for (int q = 0; q < QW; ++q) bad |= !isfinite(acc[h][q]);
+            store_cols<T>(y + h * BN, acc[h], QW);
+        }
+    }
+    if (bad) set_status(p.status, BFMOE_ERR_NONFINITE);
 }
 
 // ------------------------------------------------------ standalone rows --
