@@ -77,12 +77,12 @@ RouteLayout route_layout(int T, int N)
 }
 
 struct FwdLayout {
-    size_t status, topk_idx, gates, perm, offsets, hist, total, tiles, ntiles, coef_t, coef_p, wdec, a_blocks,
+    size_t status, topk_idx, gates, perm, offsets, hist, total, row_tok, row_exp, coef_t, coef_p, wdec, a_blocks,
         slot, total_bytes;
 };
 
 int padded_rows(int T, int k) { return (T * k + kBM - 1) / kBM * kBM; }
-int max_in_tiles(int T, int d, int N, int k) { return (T * k + tile_rows_for(d) - 1) / tile_rows_for(d) + N; }
+int in_tiles(int T, int d, int k) { return (T * k + tile_rows_for(d) - 1) / tile_rows_for(d); }
 
 FwdLayout fwd_layout(int T, int d, int N, int k)
 {
@@ -102,8 +102,8 @@ FwdLayout fwd_layout(int T, int d, int N, int k)
     l.offsets = take(((size_t)N + 1) * 4);
     l.hist = take((size_t)route_chunks(T) * N * 4);
     l.total = take((size_t)N * 4);
-    l.tiles = take((size_t)max_in_tiles(T, d, N, k) * 16);
-    l.ntiles = take(4);
+    l.row_tok = take(R * 4);
+    l.row_exp = take(R * 4);
     l.coef_t = take(ncoef * 8);
     l.coef_p = take(ncoef * 8);
     l.wdec = take((size_t)d * d * 2);
@@ -243,8 +243,10 @@ bfmoe_status launch_route(RouteParams rp, cudaStream_t st)
     const int occ = occupancy((const void *)k_route, kRouteThreads, smem);
     if (sms <= 0 || occ <= 0) return BFMOE_ERR_CUDA;
     // one block per SM at most (cheaper grid barriers), never more than the
-    // histogram holds
-    const int grid = std::min(std::min(sms, occ * sms), kMaxRouteBlocks);
+    // histogram holds, and at least 32 tokens per block (a smaller histogram
+    // to scan; the top-k of a block's tokens runs on lane groups in parallel)
+    const int by_tokens = (int)std::min<long long>(kMaxRouteBlocks, ((long long)rp.T + 31) / 32);
+    const int grid = std::max(1, std::min(std::min(std::min(sms, occ * sms), kMaxRouteBlocks), by_tokens));
     rp.skip_arrive_block = g_skip_arrive_block;
     if (launch(k_route, dim3(grid), dim3(kRouteThreads), smem, st, false, true, rp) != cudaSuccess)
         return BFMOE_ERR_CUDA;
@@ -267,8 +269,8 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     __half *wdec = reinterpret_cast<__half *>(ws + l.wdec);
     __half *ablk = reinterpret_cast<__half *>(ws + l.a_blocks);
     __half *slot = reinterpret_cast<__half *>(ws + l.slot);
-    int4 *tiles = reinterpret_cast<int4 *>(ws + l.tiles);
-    int32_t *ntiles = reinterpret_cast<int32_t *>(ws + l.ntiles);
+    int32_t *row_tok = reinterpret_cast<int32_t *>(ws + l.row_tok);
+    int32_t *row_exp = reinterpret_cast<int32_t *>(ws + l.row_exp);
     const int sms = device_sms();
     if (sms <= 0) return BFMOE_ERR_CUDA;
 
@@ -289,9 +291,8 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     rp.total = reinterpret_cast<int32_t *>(ws + l.total);
     rp.sync = status + 1;
     rp.status = status;
-    rp.in_tiles = tiles;
-    rp.n_in_tiles = ntiles;
-    rp.tile_rows = tile_rows_for(d);
+    rp.row_tok = row_tok;
+    rp.row_exp = row_exp;
     rp.d = d;
     bfmoe_status s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
@@ -308,8 +309,20 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     pp.packed = reinterpret_cast<const uint32_t *>(packed);
     pp.wdec = wdec;
     pp.status = status;
-    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, 4 * sms));
-    if (launch(k_prep, dim3(prep_grid), dim3(256), 0, st, rec == nullptr, false, pp) != cudaSuccess)
+    // one block per SM: the prep shares the SMs with the routing, whose
+    // latency chain must keep most of the issue slots
+    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, sms));
+    void (*kp)(PrepParams) = nullptr;
+    switch (L) {
+    case 6: kp = k_prep<6>; break;
+    case 7: kp = k_prep<7>; break;
+    case 8: kp = k_prep<8>; break;
+    case 9: kp = k_prep<9>; break;
+    case 10: kp = k_prep<10>; break;
+    case 11: kp = k_prep<11>; break;
+    default: kp = k_prep<12>; break;
+    }
+    if (launch(kp, dim3(prep_grid), dim3(256), 0, st, rec == nullptr, false, pp) != cudaSuccess)
         return BFMOE_ERR_CUDA;
     mark(rec, st);
 
@@ -320,20 +333,17 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     ep.k = k;
     ep.N = N;
     ep.R = R;
-    ep.perm = perm;
-    ep.tiles = tiles;
-    ep.n_tiles = ntiles;
-    ep.max_tiles = max_in_tiles(T_, d, N, k);
+    ep.row_tok = row_tok;
+    ep.row_exp = row_exp;
     ep.coef_t = ct;
-
     ep.a_blocks = ablk;
     ep.status = status;
     const bool smc = expert_in_smem_coef(d, L);
-    const size_t in_smem = expert_in_smem_bytes(d, L, smc);
+    const size_t in_smem = expert_in_smem_bytes(d, L, smc, (int)sizeof(T));
     auto kin = smc ? k_expert_in<T, true> : k_expert_in<T, false>;
     if (!ensure_smem((const void *)kin, in_smem)) return BFMOE_ERR_CUDA;
     const int in_occ = occupancy((const void *)kin, kInThreads, in_smem);
-    const int in_grid = std::max(1, std::min(max_in_tiles(T_, d, N, k), std::max(1, in_occ) * sms));
+    const int in_grid = std::max(1, std::min(in_tiles(T_, d, k), std::max(1, in_occ) * sms));
     if (launch(kin, dim3(in_grid), dim3(kInThreads), in_smem, st, true, false, ep) != cudaSuccess)
         return BFMOE_ERR_CUDA;
     mark(rec, st);
@@ -379,16 +389,30 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     const unsigned cthreads = (unsigned)T_ * (unsigned)(BN / 8);  // BN/8 threads per token
     const dim3 cgrid2((cthreads + 255) / 256);
     cudaError_t e = cudaSuccess;
+    const bool pdl = rec == nullptr;
+    const bool k2 = k == 2;
     switch (HS) {
     case 0:
-        e = BN == 256 ? launch(k_combine<T, 0, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb)
-            : BN == 128 ? launch(k_combine<T, 0, 128, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb)
-                        : launch(k_combine<T, 0, 64, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb);
+        if (BN == 256)
+            e = k2 ? launch(k_combine<T, 0, 256, 8, 2>, cgrid2, dim3(256), 0, st, pdl, false, cb)
+                   : launch(k_combine<T, 0, 256, 8, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb);
+        else if (BN == 128)
+            e = k2 ? launch(k_combine<T, 0, 128, 8, 2>, cgrid2, dim3(256), 0, st, pdl, false, cb)
+                   : launch(k_combine<T, 0, 128, 8, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb);
+        else
+            e = k2 ? launch(k_combine<T, 0, 64, 8, 2>, cgrid2, dim3(256), 0, st, pdl, false, cb)
+                   : launch(k_combine<T, 0, 64, 8, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb);
         break;
-    case 1: e = launch(k_combine<T, 1, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
-    case 2: e = launch(k_combine<T, 2, 256, 8>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
-    case 3: e = launch(k_combine<T, 3, 256, 4>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
-    default: e = launch(k_combine<T, 4, 256, 2>, cgrid2, dim3(256), 0, st, rec == nullptr, false, cb); break;
+    case 1:
+        e = k2 ? launch(k_combine<T, 1, 256, 8, 2>, cgrid2, dim3(256), 0, st, pdl, false, cb)
+               : launch(k_combine<T, 1, 256, 8, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb);
+        break;
+    case 2:
+        e = k2 ? launch(k_combine<T, 2, 256, 8, 2>, cgrid2, dim3(256), 0, st, pdl, false, cb)
+               : launch(k_combine<T, 2, 256, 8, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb);
+        break;
+    case 3: e = launch(k_combine<T, 3, 256, 4, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb); break;
+    default: e = launch(k_combine<T, 4, 256, 2, 0>, cgrid2, dim3(256), 0, st, pdl, false, cb); break;
     }
     if (e != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);
@@ -656,7 +680,7 @@ BFMOE_API int bfmoe_trace_read(unsigned long long *host, int clear)
     if (cudaDeviceSynchronize() != cudaSuccess) return BFMOE_ERR_CUDA;
     if (cudaMemcpyFromSymbol(host, g_bfmoe_trace, sizeof(g_bfmoe_trace)) != cudaSuccess) return BFMOE_ERR_CUDA;
     if (clear) {
-        static unsigned long long zeros[4][kTraceBlocks][kTraceSlots];
+        static unsigned long long zeros[kTraceKernels][kTraceBlocks][kTraceSlots];
         if (cudaMemcpyToSymbol(g_bfmoe_trace, zeros, sizeof(zeros)) != cudaSuccess) return BFMOE_ERR_CUDA;
     }
     return BFMOE_OK;

@@ -42,8 +42,9 @@ __host__ __device__ inline void pass_bounds(int L, int pi, int &s0, int &g)
 // Engine tables hold each expert's {cos a, +-sin a} in the order the
 // row engine consumes them: passes in execution order, then subsets, then
 // stages in execution order, then the subset's rotations (m ascending among
-// the indices whose local-stage bit is clear).  The sign of B^T is folded
-// in.  engine_entry gives the (stage, pair) of entry r of one expert's table.
+// the indices whose local-stage bit is clear), stored in the paired layout
+// (see rot2).  The sign of B^T is folded in.  engine_entry gives the (stage,
+// pair) of rotation r of one expert's table.
 __host__ __device__ inline void engine_entry(int d, int L, bool transpose, int r, int &s, int &p)
 {
     const int np = npass_of(L), half = d >> 1;
@@ -86,7 +87,9 @@ __host__ __device__ inline int engine_pos(int d, int L, bool transpose, int s, i
 
 // One "subset" of a row: the 2^G values whose indices differ only in bits
 // S0..S0+G-1, index base | (m << S0).  `row` is the shared-window address of
-// the row; `tab` the subset's G * 2^(G-1) table entries, read two at a time.
+// the row; `tab` the subset's G * 2^(G-1) table rotations.  Rotations ri and
+// ri+1 (ri even) of a stage above the subset's lowest bit act on the
+// adjacent pairs (m, m+1), (m+h, m+1+h): one pair instruction each.
 template <int G, int S0, bool TRANSPOSE, typename Tab>
 __device__ __forceinline__ void bfly_subset(uint32_t row, int base, Tab tab)
 {
@@ -98,39 +101,45 @@ __device__ __forceinline__ void bfly_subset(uint32_t row, int base, Tab tab)
 #pragma unroll
     for (int ql = 0; ql < G; ++ql) {
         const int ls = TRANSPOSE ? (G - 1 - ql) : ql;
-        float2 c[H];
+        const int h = 1 << ls;
 #pragma unroll
         for (int i = 0; i < H / 2; ++i) {
             const float4 w = tab.ld4(ql * H + 2 * i);
-            c[2 * i] = make_float2(w.x, w.y);
-            c[2 * i + 1] = make_float2(w.z, w.w);
-        }
-#pragma unroll
-        for (int ri = 0; ri < H; ++ri) {
-            const int m = insert_zero_bit(ri, ls);
-            const float a = v[m], b = v[m + (1 << ls)];
-            v[m] = fmaf(c[ri].x, a, -(c[ri].y * b));
-            v[m + (1 << ls)] = fmaf(c[ri].y, a, c[ri].x * b);
+            const int m0 = insert_zero_bit(2 * i, ls), m1 = insert_zero_bit(2 * i + 1, ls);
+            if (ls > 0) {
+                float2 a = make_float2(v[m0], v[m1]), b = make_float2(v[m0 + h], v[m1 + h]);
+                rot2(a, b, make_float2(w.x, w.y), make_float2(w.z, w.w));
+                v[m0] = a.x;
+                v[m1] = a.y;
+                v[m0 + h] = b.x;
+                v[m1 + h] = b.y;
+            } else {
+                rot1(v[m0], v[m0 + h], w.x, w.z);
+                rot1(v[m1], v[m1 + h], w.y, w.w);
+            }
         }
     }
 #pragma unroll
     for (int m = 0; m < M; ++m) sts_f32(row + 4u * (uint32_t)(base + (m << S0)), v[m]);
 }
 
-// One pass over `rows` rows of the tile (shared address `tile`, row stride
-// `ld` floats).  Row r uses the table  tab0 + sexp[r] * estride  (sexp ==
-// nullptr: every row uses tab0); `poff` is the pass's offset in a table.
+// One pass over the 2^lrows rows of the tile (shared address `tile`, row
+// stride `ld` floats).  Row r uses the table  tab0 + sexp[r] * estride  (sexp
+// == nullptr: every row uses tab0); `poff` is the pass's offset in a table.
+// Consecutive threads take consecutive rows of one subset, so a warp's
+// table loads are broadcasts when its rows share a table.
 template <int G, int S0, bool TRANSPOSE, typename Tab>
-__device__ __forceinline__ void bfly_pass(uint32_t tile, int ld, int rows, int d, const int *sexp, Tab tab0,
+__device__ __forceinline__ void bfly_pass(uint32_t tile, int ld, int lrows, int d, const int *sexp, Tab tab0,
                                           int estride, int poff, int nthreads)
 {
     const int nsub = d >> G;
     constexpr int S1 = S0 + G;
     constexpr int PER = G << (G - 1);
-    const int items = rows * nsub;
+    const int items = nsub << lrows;
+    const int rmask = (1 << lrows) - 1;
     for (int it = threadIdx.x; it < items; it += nthreads) {
-        const int r = it % rows;
-        const int sub = it / rows;
+        const int r = it & rmask;
+        const int sub = it >> lrows;
         const int base = ((sub >> S0) << S1) | (sub & ((1 << S0) - 1));
         const Tab tab = tab0 + ((sexp ? sexp[r] * estride : 0) + poff + sub * PER);
         bfly_subset<G, S0, TRANSPOSE>(tile + 4u * (uint32_t)(r * ld), base, tab);
@@ -138,13 +147,13 @@ __device__ __forceinline__ void bfly_pass(uint32_t tile, int ld, int rows, int d
 }
 
 template <bool TRANSPOSE, typename Tab>
-__device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, uint32_t tile, int ld, int rows, int d,
+__device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, uint32_t tile, int ld, int lrows, int d,
                                                    const int *sexp, Tab tab0, int estride, int poff)
 {
     const int nt = blockDim.x;
 #define BFLY_CASE(LL, PP, GG, SS)                                                                     \
     if (L == LL && pass == PP) {                                                                      \
-        bfly_pass<GG, SS, TRANSPOSE>(tile, ld, rows, d, sexp, tab0, estride, poff, nt);               \
+        bfly_pass<GG, SS, TRANSPOSE>(tile, ld, lrows, d, sexp, tab0, estride, poff, nt);              \
         return;                                                                                       \
     }
     BFLY_CASE(6, 0, 3, 0) BFLY_CASE(6, 1, 3, 3)
@@ -158,16 +167,15 @@ __device__ __forceinline__ void bfly_pass_dispatch(int L, int pass, uint32_t til
 }
 
 // Apply B (transpose == false) or B^T (transpose == true) to every row r <
-// rows of the shared-memory tile `tile`; row r uses the engine table (for
-// that direction) of expert sexp[r] (tables of L*d/2 entries, back to back)
+// 2^lrows of the shared-memory tile `tile`; row r uses the engine table (for
+// that direction) at tab0 + sexp[r] * estride (estride >= L*d/2 slots, even)
 // or, with sexp == nullptr, the single table tab0.  6 <= L <= 12.  Must be
 // called by all threads of the block (has __syncthreads).
 template <typename Tab>
-__device__ __forceinline__ void bfly_tile(float *tile, int ld, int rows, int d, int L, const int *sexp, Tab tab0,
-                                          bool transpose)
+__device__ __forceinline__ void bfly_tile(float *tile, int ld, int lrows, int d, int L, const int *sexp, Tab tab0,
+                                          int estride, bool transpose)
 {
     const uint32_t ts = smem_addr(tile);
-    const int estride = L * (d >> 1);
     const int np = npass_of(L);
     int poff = 0;
     for (int q = 0; q < np; ++q) {
@@ -175,15 +183,19 @@ __device__ __forceinline__ void bfly_tile(float *tile, int ld, int rows, int d, 
         int s0, g;
         pass_bounds(L, pi, s0, g);
         if (transpose)
-            bfly_pass_dispatch<true>(L, pi, ts, ld, rows, d, sexp, tab0, estride, poff);
+            bfly_pass_dispatch<true>(L, pi, ts, ld, lrows, d, sexp, tab0, estride, poff);
         else
-            bfly_pass_dispatch<false>(L, pi, ts, ld, rows, d, sexp, tab0, estride, poff);
+            bfly_pass_dispatch<false>(L, pi, ts, ld, lrows, d, sexp, tab0, estride, poff);
         poff += g * (d >> 1);
         __syncthreads();
     }
 }
 
-// Rows per shared-memory tile: up to 16, at most 16384 floats of data.
-__host__ __device__ constexpr int tile_rows_for(int d) { return (16384 / d) < 16 ? (16384 / d) : 16; }
+// log2 of a power of two.
+__host__ __device__ constexpr int ilog2_pow2(int x) { return x <= 1 ? 0 : 1 + ilog2_pow2(x >> 1); }
+
+// Rows per shared-memory tile: up to 32 (a warp's lanes), at most 16384
+// floats of data.
+__host__ __device__ constexpr int tile_rows_for(int d) { return (16384 / d) < 32 ? (16384 / d) : 32; }
 
 }  // namespace bfmoe

@@ -38,8 +38,8 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
 // boundaries: g_bfmoe_trace[kernel][block][slot] (read back with
 // bfmoe_trace_read).  Without the flag the macro compiles to nothing.
 #ifdef BFMOE_TRACE_PHASES
-constexpr int kTraceBlocks = 1024, kTraceSlots = 16;
-__device__ unsigned long long g_bfmoe_trace[4][kTraceBlocks][kTraceSlots];
+constexpr int kTraceKernels = 5, kTraceBlocks = 1024, kTraceSlots = 16;
+__device__ unsigned long long g_bfmoe_trace[kTraceKernels][kTraceBlocks][kTraceSlots];
 #define BFMOE_TRACE(kernel, cond, slot)                                                     \
     do {                                                                                    \
         if ((cond) && blockIdx.x < kTraceBlocks)                                            \
@@ -63,6 +63,10 @@ __device__ __forceinline__ void fence_barrier_init()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
 {
@@ -255,6 +259,62 @@ __device__ __forceinline__ void tmem_ld4_nowait(uint32_t taddr, float &a, float 
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ------------------------------------------------------ fp32 pairs --
+// sm_100 two-lane fp32 arithmetic (.x and .y independently, round to
+// nearest): one instruction does the work of two.
+__device__ __forceinline__ unsigned long long f2_bits(float2 v)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+__device__ __forceinline__ float2 f2_val(unsigned long long r)
+{
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b)
+{
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_val(r);
+}
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b)
+{
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_val(r);
+}
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c)
+{
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+    return f2_val(r);
+}
+
+// Cos/sin tables store their rotations in consumption order, each aligned
+// pair of rotations (2q, 2q+1) as the four floats
+// (cos_2q, cos_2q+1, sin_2q, sin_2q+1), so that one 16-byte load gives two
+// rotations in the lane layout of the pair arithmetic.  A table of n
+// rotations (n even) takes n float2 slots.
+//
+// Two Givens rotations at once, lane-wise: (a, b) <- (c a - s b, s a + c b).
+__device__ __forceinline__ void rot2(float2 &a, float2 &b, float2 c, float2 s)
+{
+    const float2 sa = f2_mul(s, a);
+    const float2 na = f2_sub(f2_mul(c, a), f2_mul(s, b));
+    b = f2_fma(c, b, sa);
+    a = na;
+}
+// One rotation: (a, b) <- (c a - s b, s a + c b).
+__device__ __forceinline__ void rot1(float &a, float &b, float c, float s)
+{
+    const float x = a, y = b;
+    a = fmaf(c, x, -(s * y));
+    b = fmaf(s, x, c * y);
+}
+
 // ------------------------------------------------ explicit shared memory --
 // Typed accesses through 32-bit shared-window addresses, so that the loads and
 // stores are shared-memory instructions whatever the compiler can prove
@@ -280,16 +340,26 @@ __device__ __forceinline__ float4 lds_f32x4(uint32_t a)
 }
 
 // A cos/sin table that lives in shared memory (address) or global memory.
+// ld4(i), i even: rotations i, i+1 as (cos_i, cos_i+1, sin_i, sin_i+1);
+// cs(i): rotation i alone as (cos, sin).
 struct SmemTab {
-    uint32_t base;  // shared-window byte address of entry 0
-    __device__ __forceinline__ float2 ld2(int i) const { return lds_f32x2(base + 8u * (uint32_t)i); }
-    __device__ __forceinline__ float4 ld4(int i) const { return lds_f32x4(base + 8u * (uint32_t)i); }  // entries i, i+1
+    uint32_t base;  // shared-window byte address of slot 0
+    __device__ __forceinline__ float4 ld4(int i) const { return lds_f32x4(base + 8u * (uint32_t)i); }
+    __device__ __forceinline__ float2 cs(int i) const
+    {
+        const uint32_t a = base + 8u * (uint32_t)(i & ~1) + 4u * (uint32_t)(i & 1);
+        return make_float2(lds_f32(a), lds_f32(a + 8u));
+    }
     __device__ __forceinline__ SmemTab operator+(int i) const { return SmemTab{base + 8u * (uint32_t)i}; }
 };
 struct GmemTab {
     const float2 *p;
-    __device__ __forceinline__ float2 ld2(int i) const { return __ldg(p + i); }
     __device__ __forceinline__ float4 ld4(int i) const { return __ldg(reinterpret_cast<const float4 *>(p + i)); }
+    __device__ __forceinline__ float2 cs(int i) const
+    {
+        const float *f = reinterpret_cast<const float *>(p + (i & ~1)) + (i & 1);
+        return make_float2(__ldg(f), __ldg(f + 2));
+    }
     __device__ __forceinline__ GmemTab operator+(int i) const { return GmemTab{p + i}; }
 };
 

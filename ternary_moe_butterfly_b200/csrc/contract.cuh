@@ -46,8 +46,16 @@ __host__ __device__ constexpr int pair_table_floats2(int BN) { return 2 * slice_
 //           ascending: 80 entries per block;
 //   pass 2: 8-column groups g, stages 5..SIN-1, columns q = 0..7, rotations
 //           over m (columns 8g + q + 32 m) with the stage's bit clear.
-// Then, for the combine, columns c < BN: stages SIN..L-1, rotations over m
-// (columns c + BN m).  out_entry gives the (stage, pair) of entry r.
+// Then, for the combine, the in-slice columns c < BN in slot order (column
+// 8g + 32m + q at slot position (g * BN/32 + m) * 8 + q, the order in which
+// the combine's threads read them): stages SIN..L-1, rotations over the
+// slices h (columns c + BN h).  out_table_entry gives the (stage, pair) of
+// entry r; out_pos is its inverse.
+__host__ __device__ constexpr int slot_col(int BN, int sp)
+{
+    return 8 * (sp / (BN / 4)) + 32 * ((sp >> 3) % (BN / 32)) + (sp & 7);
+}
+__host__ __device__ constexpr int slot_pos(int BN, int c) { return ((c >> 3) & 3) * (BN / 4) + (c >> 5) * 8 + (c & 7); }
 __host__ __device__ inline void out_table_entry(int d, int L, int r, int &s, int &p)
 {
     const int BN = gemm_bn(d), SIN = slice_stages(BN);
@@ -74,7 +82,7 @@ __host__ __device__ inline void out_table_entry(int d, int L, int r, int &s, int
     } else {
         const int w = r - NH * slice;
         const int HS = L - SIN, per = HS << (HS - 1);
-        const int c = w / per, rr = w % per;
+        const int c = slot_col(BN, w / per), rr = w % per;
         const int ls = rr >> (HS - 1);
         s = SIN + ls;
         p = pair_of(c + BN * insert_zero_bit(rr & ((1 << (HS - 1)) - 1), ls), s);
@@ -99,12 +107,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ void rot(float &a, float &b, float2 cs)
-{
-    const float x = a, y = b;
-    a = fmaf(cs.x, x, -(cs.y * y));
-    b = fmaf(cs.y, x, cs.x * y);
-}
 
 // Inverse of out_table_entry: the output-table position of (stage s, pair p).
 __host__ __device__ inline int out_pos(int d, int L, int s, int p)
@@ -122,7 +124,7 @@ __host__ __device__ inline int out_pos(int d, int L, int s, int p)
     const int HS = L - SIN, pc = HS << (HS - 1);
     const int jj = insert_zero_bit(p, s);
     const int c = jj % BN, m = jj / BN, ls = s - SIN;
-    return NH * slice + c * pc + (ls << (HS - 1)) + delete_bit(m, ls);
+    return NH * slice + slot_pos(BN, c) * pc + (ls << (HS - 1)) + delete_bit(m, ls);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
@@ -168,12 +170,22 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
         const Tab t4 = tab + blk * 80;
 #pragma unroll
         for (int s = 0; s < 5; ++s) {
+            const int h = 1 << s;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 w = t4.ld4(s * 16 + 2 * i);
                 const int m0 = insert_zero_bit(2 * i, s), m1 = insert_zero_bit(2 * i + 1, s);
-                rot(v[m0], v[m0 + (1 << s)], make_float2(w.x, w.y));
-                rot(v[m1], v[m1 + (1 << s)], make_float2(w.z, w.w));
+                if (s > 0) {  // m1 = m0 + 1: one pair instruction per rotation pair
+                    float2 a = make_float2(v[m0], v[m1]), b = make_float2(v[m0 + h], v[m1 + h]);
+                    rot2(a, b, make_float2(w.x, w.y), make_float2(w.z, w.w));
+                    v[m0] = a.x;
+                    v[m1] = a.y;
+                    v[m0 + h] = b.x;
+                    v[m1 + h] = b.y;
+                } else {
+                    rot1(v[m0], v[m0 + h], w.x, w.z);
+                    rot1(v[m1], v[m1 + h], w.y, w.w);
+                }
             }
         }
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
@@ -214,12 +226,32 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
         const Tab t2 = tab + (NB * 80 + grp * PER2);
 #pragma unroll
         for (int ls = 0; ls < G2; ++ls) {
+            const int h = 1 << ls;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
+                if constexpr (M2 >= 4) {
+                    // rotations ri, ri+1 of column q: one paired table load
 #pragma unroll
-                for (int ri = 0; ri < M2 / 2; ++ri) {
-                    const int m = insert_zero_bit(ri, ls);
-                    rot(v[q][m], v[q][m + (1 << ls)], t2.ld2((ls * 8 + q) * (M2 / 2) + ri));
+                    for (int ri = 0; ri < M2 / 2; ri += 2) {
+                        const float4 w = t2.ld4((ls * 8 + q) * (M2 / 2) + ri);
+                        const int m0 = insert_zero_bit(ri, ls), m1 = insert_zero_bit(ri + 1, ls);
+                        if (ls > 0) {
+                            float2 a = make_float2(v[q][m0], v[q][m1]), b = make_float2(v[q][m0 + h], v[q][m1 + h]);
+                            rot2(a, b, make_float2(w.x, w.y), make_float2(w.z, w.w));
+                            v[q][m0] = a.x;
+                            v[q][m1] = a.y;
+                            v[q][m0 + h] = b.x;
+                            v[q][m1 + h] = b.y;
+                        } else {
+                            rot1(v[q][m0], v[q][m0 + h], w.x, w.z);
+                            rot1(v[q][m1], v[q][m1 + h], w.y, w.w);
+                        }
+                    }
+                } else {
+                    // one rotation per column and stage: the pair partner is
+                    // the next column's
+                    const float2 cs = t2.cs((ls * 8 + q) * (M2 / 2));
+                    rot1(v[q][0], v[q][h], cs.x, cs.y);
                 }
             }
         }

@@ -66,14 +66,17 @@ __global__ void k_engine_table(const float *__restrict__ angles, int N, int d, i
                                float2 *__restrict__ out)
 {
     const int tab = L * (d / 2);
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= N * tab) return;
-    const int e = i / tab, r = i % tab;
-    int s, p;
-    engine_entry(d, L, transpose, r, s, p);
-    float sn, cs;
-    sincosf(angles[((size_t)e * L + s) * (d / 2) + p], &sn, &cs);
-    out[i] = make_float2(cs, transpose ? -sn : sn);
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;  // rotation pair
+    if (i >= N * tab / 2) return;
+    const int e = (2 * i) / tab, r = (2 * i) % tab;
+    float c[2], sn[2];
+    for (int h = 0; h < 2; ++h) {
+        int s, p;
+        engine_entry(d, L, transpose, r + h, s, p);
+        sincosf(angles[((size_t)e * L + s) * (d / 2) + p], &sn[h], &c[h]);
+        if (transpose) sn[h] = -sn[h];
+    }
+    reinterpret_cast<float4 *>(out)[i] = make_float4(c[0], c[1], sn[0], sn[1]);
 }
 
 // ------------------------------------------------------- tile row I/O --
@@ -130,107 +133,163 @@ __device__ __forceinline__ void store1(__nv_bfloat16 *dst, float v) { *dst = __f
 struct ExpertInParams {
     const void *x;
     int d, L, k, N, R;
-    const int32_t *perm;
-    const int4 *tiles;       // single-expert row tiles {expert, row0, nrows, -}
-    const int32_t *n_tiles;
-    int max_tiles;           // capacity of `tiles`
+    const int32_t *row_tok;  // [R] token of each bucket row
+    const int32_t *row_exp;  // [R] expert of each bucket row
     const float2 *coef_t;    // [N][L*d/2] engine table of theta (B^T order)
     __half *a_blocks;        // fp16 operand blocks, rows in bucket order
     uint32_t *status;
 };
 
-// Persistent over the tile list: gather the rows of one expert's tile, rotate
-// by B(theta_e)^T (the expert's cos/sin table is staged in shared memory when
-// it fits, so every coefficient load is a broadcast), write fp16 A blocks.
-constexpr int kInThreads = 128;  // four CTAs per SM
+// Persistent over tiles of tile_rows_for(d) consecutive bucket rows (one
+// lane per row at d <= 512): gather the rows, rotate each by B(theta_e)^T of
+// its own expert, write fp16 A blocks.  A tile holds the ends of at most a
+// few buckets: when its rows have at most two experts, both experts'
+// cos/sin tables are staged in shared memory (16 bytes apart in bank terms,
+// so the two addresses of a warp's table load fall in distinct banks), else
+// the rows read their tables from global memory.  Rows and tables arrive by
+// bulk copies on one mbarrier (one memory latency per tile); the raw rows
+// land in the fp32 tile's own bytes and are widened in place, in row groups
+// whose order never overwrites raw data that is still to be read.
+constexpr int kInThreads = 256;  // two CTAs per SM
+
+// Byte stride of a raw staged row: 16 bytes of padding put the rows' 16-byte
+// chunks in distinct bank groups for the lanes-are-rows widening loads.
+__host__ __device__ constexpr uint32_t raw_row_stride(int d, int esize) { return (uint32_t)(d * esize + 16); }
+// Shared-memory stride between the two staged tables, in entries.
+__host__ __device__ constexpr int staged_table_stride(int d, int L) { return L * (d >> 1) + 2; }
 
 template <typename T, bool SMEM_COEF>
-__global__ void __launch_bounds__(kInThreads, 4) k_expert_in(ExpertInParams p)
+__global__ void __launch_bounds__(kInThreads, 2) k_expert_in(ExpertInParams p)
 {
-    extern __shared__ __align__(16) float smem_f[];
+    extern __shared__ __align__(16) uint8_t smem_in[];
     const int d = p.d, L = p.L;
     const int RT = tile_rows_for(d);
     const int ld = d + 1;
-    const size_t tab = (size_t)L * (d >> 1);
-    float2 *sc = reinterpret_cast<float2 *>(smem_f);  // [tab] when SMEM_COEF
-    float *tile = smem_f + (SMEM_COEF ? 2 * tab : 0);
-    int *stok = reinterpret_cast<int *>(tile + (size_t)RT * ld);
+    const int tab = L * (d >> 1);
+    const int tstride = staged_table_stride(d, L);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem_in);
+    int *mode = reinterpret_cast<int *>(smem_in + 8);    // 1: this tile's tables are staged
+    int *stok = reinterpret_cast<int *>(smem_in + 16);   // [32] token of each tile row, -1: none
+    int *sexp = reinterpret_cast<int *>(smem_in + 144);  // [32] table index of each tile row
+    float2 *sc = reinterpret_cast<float2 *>(smem_in + 272);  // [2][tstride] when SMEM_COEF
+    uint8_t *region = smem_in + 272 + (SMEM_COEF ? (size_t)2 * tstride * 8 : 0);
+    float *tile = reinterpret_cast<float *>(region);  // [RT][ld] fp32, raw rows land here first
+    constexpr int VPC = 16 / sizeof(T);                 // values per 16-byte chunk
+    const uint32_t rs = raw_row_stride(d, sizeof(T));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
     BFMOE_TRACE(1, threadIdx.x == 0, 0);
     pdl_wait();
     pdl_trigger();
     BFMOE_TRACE(1, threadIdx.x == 0, 1);
-    // a routing that gave up (timeout) leaves the list unspecified: clamp it
-    const int ntiles = min(max(*p.n_tiles, 0), p.max_tiles);
     const T *x = reinterpret_cast<const T *>(p.x);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int KC = d / kBK;
+    const int nchunk = d / VPC;  // 16-byte chunks per row
+    const int ntiles = (p.R + RT - 1) / RT;
+    const int T_ = p.R / p.k;
+    // rows widened per group: at most 8 chunks in flight per thread
+    const int grows = max(1, min(RT, 8 * kInThreads / nchunk));
+    uint32_t phase = 0;
     for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
-        const int4 tl = p.tiles[ti];
-        const int e = min(max(tl.x, 0), p.N - 1);
-        const int r0 = tl.y;
-        int nr = min(max(tl.z, 0), RT);
-        if (r0 < 0 || r0 > p.R - nr) nr = 0;
-        if (nr == 0) continue;  // uniform across the block
-        const float2 *gtab = p.coef_t + (size_t)e * tab;
+        const int r0 = ti * RT;
+        const int nr = min(RT, p.R - r0);
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 5);
-        if ((int)threadIdx.x < RT) {
-            int t = -1;
-            const int r = r0 + (int)threadIdx.x;
-            if ((int)threadIdx.x < nr && r >= 0 && r < p.R) {
-                const int i = p.perm[r];
-                if (i >= 0 && i < p.R) t = i / p.k;
+        if (warp == 0) {
+            // the rows' tokens and experts: one memory latency
+            int t = -1, e = 0;
+            if (lane < nr) {
+                t = p.row_tok[r0 + lane];
+                e = p.row_exp[r0 + lane];
+                if (t < 0 || t >= T_) t = -1;
+                if (e < 0 || e >= p.N) {
+                    e = 0;
+                    t = -1;
+                }
             }
-            stok[threadIdx.x] = t;
+            const int ea = __shfl_sync(0xffffffffu, e, 0), eb = __shfl_sync(0xffffffffu, e, nr - 1);
+            const bool two = SMEM_COEF && __all_sync(0xffffffffu, lane >= nr || e == ea || e == eb);
+            if (lane < RT) {
+                stok[lane] = t;
+                sexp[lane] = two ? (e == ea ? 0 : 1) : e;
+            }
+            const unsigned have = __ballot_sync(0xffffffffu, t >= 0);
+            if (lane == 0) {
+                // the previous tile's reads of this memory (generic proxy)
+                // come before the bulk copies' writes (async proxy)
+                fence_proxy_async_smem();
+                const uint32_t tb = (uint32_t)tab * 8;
+                const uint32_t bytes = (uint32_t)__popc(have) * (uint32_t)(d * sizeof(T)) +
+                                       (two ? (ea == eb ? tb : 2 * tb) : 0u);
+                mbar_arrive_expect_tx(bar, bytes);
+                if (two) {
+                    bulk_g2s(sc, p.coef_t + (size_t)ea * tab, tb, bar);
+                    if (eb != ea) bulk_g2s(sc + tstride, p.coef_t + (size_t)eb * tab, tb, bar);
+                }
+            }
+            __syncwarp();
+            if (t >= 0) {
+                fence_proxy_async_smem();
+                bulk_g2s(region + (size_t)lane * rs, x + (size_t)t * d, (uint32_t)(d * sizeof(T)), bar);
+            }
+            if (lane == 0) *mode = two ? 1 : 0;
         }
-        __syncthreads();
-        // gather: lane = tile row, warp = 16-byte column chunk, so the scalar
-        // shared-memory stores of a warp hit 32 distinct banks; the first
-        // batch of loads is issued before the expert's table is built, so
-        // the two overlap
+        const bool ok = __syncthreads_and(mbar_wait(bar, phase));
+        phase ^= 1;
+        if (!ok) {
+            if (threadIdx.x == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
+            break;
+        }
+        const bool two = *mode != 0;
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 6);
-        const int t_lane = lane < nr ? stok[lane] : -1;
-        constexpr int VPC = 16 / sizeof(T);  // values per 16-byte chunk
-        const int nchunk = d / VPC;
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(t_lane >= 0 ? t_lane : 0) * d);
-        float *dst = tile + (size_t)lane * ld;
-        for (int c0 = warp; c0 < nchunk; c0 += 8 * nw) {
+        // widen raw -> fp32 rows in place: 2-byte types from the last group
+        // down (an fp32 row starts at or beyond twice its raw row's offset),
+        // 4-byte types from the first group up (a raw row is the longer one)
+        const int ngr = (nr + grows - 1) / grows;
+        for (int gi = 0; gi < ngr; ++gi) {
+            const int g = sizeof(T) == 2 ? ngr - 1 - gi : gi;
+            const int ra = g * grows, rn = min(grows, nr - ra);
             uint4 u[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int c = c0 + q * nw;
-                u[q] = (t_lane >= 0 && c < nchunk) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            for (int w = 0; w < 8; ++w) {
+                const int q = (int)threadIdx.x + w * kInThreads;
+                const int rr = q % rn, c = q / rn;
+                u[w] = make_uint4(0, 0, 0, 0);
+                if (c < nchunk && stok[ra + rr] >= 0)
+                    u[w] = *reinterpret_cast<const uint4 *>(region + (size_t)(ra + rr) * rs + (size_t)c * 16);
             }
-            if (SMEM_COEF && c0 == warp) {
-                // stage the expert's table (contiguous) while the row loads fly
-                copy_g2s(reinterpret_cast<const float4 *>(gtab), reinterpret_cast<float4 *>(sc), (int)tab / 2,
-                         threadIdx.x, blockDim.x);
-                BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 7);
-            }
-            if (lane < nr) {
+            __syncthreads();
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int c = c0 + q * nw;
-                    if (c >= nchunk) break;
-                    float f[8];
-                    if (VPC == 8) {
-                        unpack_bf16x8(u[q], f);
-                    } else {
-                        f[0] = __uint_as_float(u[q].x);
-                        f[1] = __uint_as_float(u[q].y);
-                        f[2] = __uint_as_float(u[q].z);
-                        f[3] = __uint_as_float(u[q].w);
-                    }
-#pragma unroll
-                    for (int i = 0; i < VPC; ++i) dst[c * VPC + i] = f[i];
+            for (int w = 0; w < 8; ++w) {
+                const int q = (int)threadIdx.x + w * kInThreads;
+                const int rr = q % rn, c = q / rn;
+                if (c >= nchunk) break;
+                float f[VPC];
+                if constexpr (VPC == 8) {
+                    unpack_bf16x8(u[w], f);
+                } else {
+                    f[0] = __uint_as_float(u[w].x);
+                    f[1] = __uint_as_float(u[w].y);
+                    f[2] = __uint_as_float(u[w].z);
+                    f[3] = __uint_as_float(u[w].w);
                 }
+                float *dst = tile + (size_t)(ra + rr) * ld + c * VPC;
+#pragma unroll
+                for (int i = 0; i < VPC; ++i) dst[i] = f[i];
             }
         }
         __syncthreads();
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 3);
-        if (SMEM_COEF)
-            bfly_tile(tile, ld, nr, d, L, nullptr, SmemTab{smem_addr(sc)}, /*transpose=*/true);
+        // all RT rows go through the engine (rows past nr hold stale values
+        // and are never stored): a power-of-two row count maps threads to
+        // rows with masks
+        if (two)
+            bfly_tile(tile, ld, ilog2_pow2(RT), d, L, sexp, SmemTab{smem_addr(sc)}, tstride, /*transpose=*/true);
         else
-            bfly_tile(tile, ld, nr, d, L, nullptr, GmemTab{gtab}, /*transpose=*/true);
+            bfly_tile(tile, ld, ilog2_pow2(RT), d, L, sexp, GmemTab{p.coef_t}, tab, /*transpose=*/true);
         BFMOE_TRACE(1, threadIdx.x == 0 && ti == (int)blockIdx.x, 4);
         bool overflow = false;
         const int nch = nr * (d / 8);
@@ -252,15 +311,16 @@ __global__ void __launch_bounds__(kInThreads, 4) k_expert_in(ExpertInParams p)
     BFMOE_TRACE(1, threadIdx.x == 0, 2);
 }
 
-__host__ inline size_t expert_in_smem_bytes(int d, int L, bool smem_coef)
+__host__ inline size_t expert_in_smem_bytes(int d, int L, bool smem_coef, int esize)
 {
-    const int RT = tile_rows_for(d);
-    return (smem_coef ? (size_t)L * (d / 2) * 8 : 0) + (size_t)RT * (d + 1) * 4 + (size_t)RT * 4;
+    const size_t RT = tile_rows_for(d);
+    const size_t raw = RT * raw_row_stride(d, esize), wide = RT * (size_t)(d + 1) * 4;
+    return 272 + (smem_coef ? (size_t)2 * staged_table_stride(d, L) * 8 : 0) + (raw > wide ? raw : wide);
 }
 
-__host__ inline bool expert_in_smem_coef(int d, int L) { return (size_t)L * (d / 2) * 8 <= 40 * 1024; }
-
-// ------------------------------------------------------------ combine --
+// Whether tiles may stage their experts' tables in shared memory: two
+// tables of up to 20 KB.
+__host__ inline bool expert_in_smem_coef(int d, int L) { return (size_t)L * (d / 2) * 8 <= 20 * 1024; }
 
 // Slot layout.  The contraction epilogue leaves each routed row i = t*k + j
 // as alpha * g_{t,j} * (output butterfly stages 0 .. SIN-1 applied), fp16,
@@ -322,12 +382,27 @@ __device__ __forceinline__ void load_halves(const __half *src, float *f)
     }
 }
 
+// n consecutive table entries (n even, 16-byte aligned) as n/2 16-byte loads
+template <int n>
+__device__ __forceinline__ void load_coef(const float2 *src, float2 *w)
+{
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+        const float4 f = __ldg(reinterpret_cast<const float4 *>(src) + i);
+        w[2 * i] = make_float2(f.x, f.y);
+        w[2 * i + 1] = make_float2(f.z, f.w);
+    }
+}
+
 // y_t = sum_j (stages s_lo..L-1 of B(phi_e)) slot_{t,j}: the rows arrive
 // already scaled by alpha * g.  HS = L - s_lo stages mix the NH = 2^HS slices
 // (pairs of slices nh, nh + 2^ls at the same in-slice column).  One thread per
 // (token, 8-column group, m) handles QW of the group's 8 columns per round in
-// all NH slices; the k rows are summed in j order.
-template <typename T, int HS, int BN, int QW>
+// all NH slices; the k rows are summed in j order.  KC > 0 fixes k = KC at
+// compile time and issues the loads of all k rows together (expert indices,
+// then rows and tables: two memory latencies per token); KC = 0 takes k from
+// the parameters, one row at a time.
+template <typename T, int HS, int BN, int QW, int KC>
 __global__ void __launch_bounds__(256) k_combine(CombineParams p)
 {
     BFMOE_TRACE(3, threadIdx.x == 0, 0);
@@ -338,9 +413,11 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
     constexpr int M2 = BN / 32;
     constexpr int TPT = 4 * M2;  // threads per token
     constexpr int PC = HS > 0 ? (HS << (HS - 1)) : 1;  // table entries per column
+    constexpr int KB = KC > 0 ? KC : 1;                 // rows loaded together
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     const int t = tid / TPT;
     if (t >= p.T) return;
+    const int k = KC > 0 ? KC : p.k;
     const int g = (tid % TPT) / M2, m = tid % M2;
     const int d = p.d, half = d >> 1;
     const int col0 = 8 * g + 32 * m;           // first of the thread's 8 in-slice columns
@@ -354,35 +431,59 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
 #pragma unroll
             for (int q = 0; q < QW; ++q) acc[h][q] = 0.0f;
 #pragma unroll 1
-        for (int j = 0; j < p.k; ++j) {
-            const int i = t * p.k + j;
-            const __half *row = p.slot + (size_t)i * d + pos0 + q0;
-            float v[NH][QW];
+        for (int j0 = 0; j0 < k; j0 += KB) {
+            float v[KB][NH][QW];
+            int ev[KB];
 #pragma unroll
-            for (int h = 0; h < NH; ++h) load_halves<QW>(row + h * BN, v[h]);
-            if (HS > 0) {
-                const int e = min(max(p.topk_idx[i], 0), p.N - 1);
-                // combine part of the output table: [column][ls][pair over slices]
-                const float2 *cf = p.coef_p + (size_t)e * p.L * half + (size_t)p.s_lo * half;
+            for (int b = 0; b < KB; ++b) {
+                const int i = t * k + j0 + b;
+                ev[b] = HS > 0 ? min(max(__ldg(p.topk_idx + i), 0), p.N - 1) : 0;
+                const __half *row = p.slot + (size_t)i * d + pos0 + q0;
 #pragma unroll
-                for (int q = 0; q < QW; ++q) {
-                    const float2 *cq = cf + (size_t)(col0 + q0 + q) * PC;
-#pragma unroll
-                    for (int ls = 0; ls < HS; ++ls)
-#pragma unroll
-                        for (int ri = 0; ri < NH / 2; ++ri) {
-                            const int h = insert_zero_bit(ri, ls);
-                            const float2 w = __ldg(cq + (ls << (HS > 0 ? HS - 1 : 0)) + ri);
-                            const float a = v[h][q], b = v[h + (1 << ls)][q];
-                            v[h][q] = fmaf(w.x, a, -(w.y * b));
-                            v[h + (1 << ls)][q] = fmaf(w.y, a, w.x * b);
-                        }
-                }
+                for (int h = 0; h < NH; ++h) load_halves<QW>(row + h * BN, v[b][h]);
             }
 #pragma unroll
-            for (int h = 0; h < NH; ++h)
+            for (int b = 0; b < KB; ++b) {
+                if (HS > 0) {
+                    // combine part of the output table: [slot position][ls][pair over slices]
+                    const float2 *cf = p.coef_p + (size_t)ev[b] * p.L * half + (size_t)p.s_lo * half;
+                    if constexpr (PC == 1) {
+                        // one rotation per column: columns q, q+1 as a pair
+                        float2 w[QW];
+                        load_coef<QW>(cf + pos0 + q0, w);
 #pragma unroll
-                for (int q = 0; q < QW; ++q) acc[h][q] += v[h][q];
+                        for (int q = 0; q < QW; q += 2) {
+                            float2 a = make_float2(v[b][0][q], v[b][0][q + 1]);
+                            float2 c = make_float2(v[b][1][q], v[b][1][q + 1]);
+                            rot2(a, c, w[q], w[q + 1]);
+                            v[b][0][q] = a.x;
+                            v[b][0][q + 1] = a.y;
+                            v[b][1][q] = c.x;
+                            v[b][1][q + 1] = c.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < QW; ++q) {
+                            float2 w[PC];
+                            load_coef<PC>(cf + (size_t)(pos0 + q0 + q) * PC, w);
+                            const float *wf = reinterpret_cast<const float *>(w);
+#pragma unroll
+                            for (int ls = 0; ls < HS; ++ls)
+#pragma unroll
+                                for (int ri = 0; ri < NH / 2; ++ri) {
+                                    const int h = insert_zero_bit(ri, ls);
+                                    const int r = (ls << (HS > 0 ? HS - 1 : 0)) + ri;
+                                    rot1(v[b][h][q], v[b][h + (1 << ls)][q], wf[4 * (r >> 1) + (r & 1)],
+                                         wf[4 * (r >> 1) + 2 + (r & 1)]);
+                                }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+#pragma unroll
+                    for (int q = 0; q < QW; ++q) acc[h][q] += v[b][h][q];
+            }
         }
         T *y = reinterpret_cast<T *>(p.y) + (size_t)t * d + col0 + q0;
 #pragma unroll
@@ -393,6 +494,7 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
         }
     }
     if (bad) set_status(p.status, BFMOE_ERR_NONFINITE);
+    BFMOE_TRACE(3, (threadIdx.x & 31) == 0, 2);
 }
 
 // ------------------------------------------------------ standalone rows --
@@ -429,7 +531,7 @@ __global__ void __launch_bounds__(256) k_bfly_apply(const T *__restrict__ x, int
             for (int c = lane; c < d; c += 32) dst[c] = 0.0f;
     }
     __syncthreads();
-    bfly_tile(tile, ld, RT, d, L, sexp, GmemTab{coef}, transpose != 0);
+    bfly_tile(tile, ld, ilog2_pow2(RT), d, L, sexp, GmemTab{coef}, L * (d >> 1), transpose != 0);
     const int nch = nr * (d / 8);
     for (int q = threadIdx.x; q < nch; q += blockDim.x) {
         const int rq = q / (d / 8), c8 = q % (d / 8);

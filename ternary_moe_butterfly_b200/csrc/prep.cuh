@@ -33,49 +33,64 @@ struct PrepParams {
 // position order, so each table line is written whole by one warp, and
 // gather their angles (the kernels that read the tables right after run
 // faster from lines that were not assembled from many SMs' partial writes).
+// Instantiated per L = log2 d, so that the index decoding divides by
+// compile-time constants.
+template <int LL>
 __global__ void __launch_bounds__(256) k_prep(PrepParams p)
 {
-    const int d = p.d, L = p.L, half = d >> 1;
-    const int tab = L * half;
+    // the input-butterfly kernel may become resident now; it still waits for
+    // this grid (and so for the routing) to complete before reading anything
+    BFMOE_TRACE(4, threadIdx.x == 0, 0);
+    pdl_trigger();
+    constexpr int L = LL, d = 1 << LL, half = d >> 1;
+    constexpr int tab = L * half;
     const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
     const int gthreads = gridDim.x * blockDim.x;
-    const int total = 2 * p.ncoef;
-    for (int i0 = gtid; i0 < total; i0 += 4 * gthreads) {
-        float a[4];
-        int dst[4];
+    // rotation pairs: [0, ncoef/2) of the input table, then the output table
+    const int npair = p.ncoef;
+    for (int j0 = gtid; j0 < npair; j0 += 2 * gthreads) {
+        float a[2][2];
+        int dst[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * gthreads;
+        for (int u = 0; u < 2; ++u) {
+            const int j = j0 + u * gthreads;
             dst[u] = -1;
-            a[u] = 0.0f;
-            if (i < total) {
-                const bool out = i >= p.ncoef;
-                const int j = out ? i - p.ncoef : i;
-                const int e = j / tab, r = j - e * tab;
-                int st, pp;
-                if (out)
-                    out_table_entry(d, L, r, st, pp);
-                else
-                    engine_entry(d, L, true, r, st, pp);
-                a[u] = __ldg((out ? p.phi : p.theta) + (size_t)e * tab + st * half + pp);
-                dst[u] = i;
+            a[u][0] = a[u][1] = 0.0f;
+            if (j < npair) {
+                const bool out = j >= p.ncoef / 2;
+                const int jj = out ? j - p.ncoef / 2 : j;
+                const int e = (2 * jj) / tab, r = (2 * jj) % tab;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    int st, pp;
+                    if (out)
+                        out_table_entry(d, L, r + h, st, pp);
+                    else
+                        engine_entry(d, L, true, r + h, st, pp);
+                    a[u][h] = __ldg((out ? p.phi : p.theta) + (size_t)e * tab + st * half + pp);
+                }
+                dst[u] = j;
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2; ++u) {
             if (dst[u] < 0) continue;
-            float sn, cs;
-            __sincosf(a[u], &sn, &cs);
-            if (dst[u] >= p.ncoef)
-                p.coef_p[dst[u] - p.ncoef] = make_float2(cs, sn);
+            float s0, c0, s1, c1;
+            __sincosf(a[u][0], &s0, &c0);
+            __sincosf(a[u][1], &s1, &c1);
+            if (dst[u] >= p.ncoef / 2)
+                reinterpret_cast<float4 *>(p.coef_p)[dst[u] - p.ncoef / 2] = make_float4(c0, c1, s0, s1);
             else
-                p.coef_t[dst[u]] = make_float2(cs, -sn);
+                reinterpret_cast<float4 *>(p.coef_t)[dst[u]] = make_float4(c0, c1, -s0, -s1);
         }
     }
+    BFMOE_TRACE(4, threadIdx.x == 0, 1);
     if (gtid == 0 && (p.packed[0] != kPackMagic || p.packed[1] != (uint32_t)d)) set_status(p.status, BFMOE_ERR_INVALID_ARG);
-    const int nq = d * d / 8;
+    constexpr int nq = d * d / 8;
     for (int q = gtid; q < nq; q += gthreads) decode_chunk(p.packed, d, p.wdec, q);
+    BFMOE_TRACE(4, threadIdx.x == 0, 2);
     pdl_wait();  // complete only after the routing has
+    BFMOE_TRACE(4, threadIdx.x == 0, 3);
 }
 
 }  // namespace bfmoe

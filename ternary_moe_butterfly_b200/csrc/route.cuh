@@ -10,17 +10,17 @@
 // Phases, separated by one or two bounded grid barriers (all blocks are
 // co-resident: the kernel is launched cooperatively):
 //   A  each block takes a contiguous token range; batches of its tokens'
-//      logits are staged in shared memory and one thread (one warp beyond
-//      256 experts) per token selects the top-k; the block counts its rows
-//      per expert (hist[block][e]).
-//   B  up to 512 experts, every block reads the (expert-major) histogram
-//      and forms the expert totals and its own prefix over the blocks before
-//      it; beyond, one warp per expert scans the column over the blocks and a
+//      logits are staged in shared memory and a group of lanes per token
+//      selects the top-k; the block counts its rows per expert
+//      (hist[block][e]) and keeps its rows' experts in shared memory.
+//   B  up to 512 experts, every block reads the block-major histogram and
+//      forms the expert totals and its own prefix over the blocks before it;
+//      beyond, one warp per expert scans the column over the blocks and a
 //      second grid barrier publishes the prefixes.
-//   C  every block scans the expert totals into bucket offsets, then ranks
-//      the rows of its tokens inside their buckets (warp match + popcount)
-//      and scatters perm / row_pos; the blocks also write the list of
-//      single-expert row tiles that the input-butterfly kernel walks.
+//   C  one warp per block scans the expert totals into bucket offsets, then
+//      ranks the rows of the block's tokens inside their buckets (warp match
+//      + popcount) and scatters perm / row_pos, and for the forward the
+//      token and expert of every bucket row.
 #pragma once
 
 #include "butterfly.cuh"
@@ -38,7 +38,6 @@ constexpr int kRouteThreads = 256;
 constexpr int kMaxK = 8;
 constexpr int kMaxRouteBlocks = 512;  // capacity of the per-block histogram
 constexpr int kOneBarrierMaxN = 512;  // up to this many experts the routing needs one grid barrier
-constexpr int kHistStageInts = 8192;  // histogram ints staged per chunk (32 KB)
 constexpr uint32_t kPackMagic = 0x32574642u;  // "BFW2"
 
 __host__ __device__ constexpr int gemm_bn(int d) { return d < 256 ? d : 256; }
@@ -58,20 +57,26 @@ struct RouteParams {
     uint32_t *status;
     int skip_arrive_block;  // test hook: this block never reaches barrier 1 (-1: none)
     int d;
-    // forward only: single-expert row tiles for the input butterfly
-    int4 *in_tiles;
-    int32_t *n_in_tiles;
-    int tile_rows;
+    // forward only: the bucket rows' tokens and experts for the input butterfly
+    int32_t *row_tok;    // [T*k] token of each bucket row, or null
+    int32_t *row_exp;    // [T*k] expert of each bucket row, or null
 };
 
-// Up to this many experts one thread selects a token's top-k.
-constexpr int kThreadTopkMaxN = 256;
+// Histogram budget of the route kernel's shared memory, and the number of
+// selected experts of its own rows a block keeps for the scatter.
+constexpr int kSelCap = 2048;
+constexpr int kLogitStageInts = 10240;  // staged logits per batch (40 KB)
 
-// Tokens staged per batch: one per thread (at most 256), at most ~40 KB of
-// logits.
+// Padded shared-memory row of one token's logits when `grp` lanes share
+// the token: rows G floats apart on top of a 32-float multiple put the group's
+// reads on distinct banks.
+__host__ __device__ inline int logit_row_stride(int N, int grp) { return grp < 32 ? ((N + 31) & ~31) + grp : N; }
+
+// Tokens staged per batch: at most 256 and what the staging area holds at
+// the widest row stride (16 lanes per token).
 __host__ __device__ inline int route_batch_tokens(int N)
 {
-    const int b = (40 * 1024 / 4) / (N + 1);
+    const int b = kLogitStageInts / logit_row_stride(N, 16);
     return b < 1 ? 1 : (b > 256 ? 256 : b);
 }
 
@@ -136,10 +141,37 @@ __device__ __forceinline__ void gates_of(const float *val, int k, float *g)
     }
 }
 
-// Top-k of one token by one thread: a sorted list of the K best (value,
-// index) pairs in registers, one pass over the N logits at stride `stride`.
+// Insert (v, e) into the sorted list of the K best (value, index) pairs.
 template <int K>
-__device__ __forceinline__ void topk_thread(const RouteParams &p, int t, const float *l, int *sh_hist)
+__device__ __forceinline__ void topk_insert(float (&val)[K], int (&sel)[K], float v, int e)
+{
+    bool b[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) b[j] = ranks_before(v, e, val[j], sel[j]);
+#pragma unroll
+    for (int j = K - 1; j > 0; --j) {
+        if (b[j]) {
+            val[j] = b[j - 1] ? val[j - 1] : v;
+            sel[j] = b[j - 1] ? sel[j - 1] : e;
+        }
+    }
+    if (b[0]) {
+        val[0] = v;
+        sel[0] = e;
+    }
+}
+
+// Top-K of one token by a group of `grp` lanes (a power of two <= 32,
+// aligned inside the warp): lane s of the group keeps the sorted K best of
+// experts s, s + grp, ...; the lists are merged across the group with xor
+// shuffles (every lane of the warp takes part; `active` only gates the scan
+// and the writes).  The order is total (value, then index), so the merged
+// list is the exact top-K whatever the scan order.  Lane 0 of the group
+// writes the indices and gates, counts the rows in the block histogram and
+// keeps the indices in `keep` (when non-null).
+template <int K>
+__device__ __forceinline__ void topk_group(const RouteParams &p, int t, const float *l, int s, int grp, bool active,
+                                           int *sh_hist, int *keep)
 {
     float val[K];
     int sel[K];
@@ -148,96 +180,49 @@ __device__ __forceinline__ void topk_thread(const RouteParams &p, int t, const f
         val[j] = -INFINITY;
         sel[j] = 0x7fffffff;  // ranks after every real candidate
     }
-    for (int e = 0; e < p.N; ++e) {
-        const float v = l[e];
-        bool b[K];
+    if (active)
+        for (int e = s; e < p.N; e += grp) topk_insert<K>(val, sel, l[e], e);
+    for (int off = 1; off < grp; off <<= 1) {
+        float ov[K];
+        int oe[K];
 #pragma unroll
-        for (int j = 0; j < K; ++j) b[j] = ranks_before(v, e, val[j], sel[j]);
+        for (int j = 0; j < K; ++j) {
+            ov[j] = __shfl_xor_sync(0xffffffffu, val[j], off);
+            oe[j] = __shfl_xor_sync(0xffffffffu, sel[j], off);
+        }
 #pragma unroll
-        for (int j = K - 1; j > 0; --j) {
-            if (b[j]) {
-                val[j] = b[j - 1] ? val[j - 1] : v;
-                sel[j] = b[j - 1] ? sel[j - 1] : e;
-            }
-        }
-        if (b[0]) {
-            val[0] = v;
-            sel[0] = e;
-        }
+        for (int j = 0; j < K; ++j) topk_insert<K>(val, sel, ov[j], oe[j]);
     }
-    float g[K];
-    gates_of(val, K, g);
+    if (active && s == 0) {
+        float g[K];
+        gates_of(val, K, g);
 #pragma unroll
-    for (int j = 0; j < K; ++j) {
-        p.topk_idx[(size_t)t * K + j] = sel[j];
-        p.gates[(size_t)t * K + j] = g[j];
-        atomicAdd(&sh_hist[sel[j]], 1);
-    }
-}
-
-// Top-k and gates of one token whose N logits are in shared memory (NaN
-// already replaced by -inf); one warp.  Lane 0 writes the results and counts
-// the token's rows in the block histogram.
-__device__ __forceinline__ void topk_token(const RouteParams &p, int t, const float *l, int *sh_hist)
-{
-    const int N = p.N, k = p.k;
-    const int lane = threadIdx.x & 31;
-    int sel[kMaxK];
-    float val[kMaxK];
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-        if (j >= k) break;
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
-        for (int e = lane; e < N; e += 32) {
-            bool taken = false;
-#pragma unroll
-            for (int jj = 0; jj < kMaxK; ++jj)
-                if (jj < j) taken |= (sel[jj] == e);
-            if (taken) continue;
-            const float v = l[e];
-            if (be == 0x7fffffff || ranks_before(v, e, bv, be)) {
-                bv = v;
-                be = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (oe != 0x7fffffff && (be == 0x7fffffff || ranks_before(ov, oe, bv, be))) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        sel[j] = be;
-        val[j] = bv;
-    }
-    if (lane == 0) {
-        float g[kMaxK];
-        gates_of(val, k, g);
-        for (int j = 0; j < k; ++j) {
-            p.topk_idx[(size_t)t * k + j] = sel[j];
-            p.gates[(size_t)t * k + j] = g[j];
+        for (int j = 0; j < K; ++j) {
+            p.topk_idx[(size_t)t * K + j] = sel[j];
+            p.gates[(size_t)t * K + j] = g[j];
             atomicAdd(&sh_hist[sel[j]], 1);
+            if (keep) keep[j] = sel[j];
         }
     }
 }
 
 // Top-k, gates and the histogram of the block's token range [t0, t1).
 // Batches of tokens are staged in shared memory with coalesced 16-byte loads
-// (one memory latency per batch; NaN becomes -inf and is reported).  Up to
-// kThreadTopkMaxN experts one thread selects for one token (rows padded to
-// N+1 floats so the threads' column reads hit distinct banks); beyond, one
-// warp per token.
-__device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, float *sh_logits, bool &saw_nan)
+// (one memory latency per batch; NaN becomes -inf and is reported); a group
+// of lanes (as many as 256 threads allow per staged token, up to a warp)
+// selects each token's experts.  `keep` (or null) receives the selected
+// experts of the range's rows in row order.
+__device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, float *sh_logits, int *keep,
+                           bool &saw_nan)
 {
     const int N = p.N;
-    const bool per_thread = N <= kThreadTopkMaxN;
-    const int ldl = per_thread ? N + 1 : N;
-    const int batch = route_batch_tokens(N);
+    const int want = max(1, min(t1 - t0, route_batch_tokens(N)));
+    int grp = 1;
+    while (grp < 32 && 2 * grp * want <= (int)blockDim.x) grp <<= 1;
+    const int batch = min(want, (int)blockDim.x / grp);
+    const int ldl = logit_row_stride(N, grp);
     for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
-    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int q = threadIdx.x / grp, s = threadIdx.x % grp;
     for (int b0 = t0; b0 < t1; b0 += batch) {
         const int nb = min(batch, t1 - b0);
         const size_t nval = (size_t)nb * N;
@@ -250,15 +235,15 @@ __device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, f
                 float4 v[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int q = q0 + u * blockDim.x;
-                    if (q < n4) v[u] = __ldg(s4 + q);
+                    const int qq = q0 + u * blockDim.x;
+                    if (qq < n4) v[u] = __ldg(s4 + qq);
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int q = q0 + u * blockDim.x;
-                    if (q >= n4) break;
+                    const int qq = q0 + u * blockDim.x;
+                    if (qq >= n4) break;
                     const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                    const int tok = (4 * q) / N, e0 = (4 * q) % N;
+                    const int tok = (4 * qq) / N, e0 = (4 * qq) % N;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         float xv = f[i];
@@ -271,33 +256,32 @@ __device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, f
                 }
             }
         } else {
-            for (size_t q = threadIdx.x; q < nval; q += blockDim.x) {
-                float xv = __ldg(src + q);
+            for (size_t qq = threadIdx.x; qq < nval; qq += blockDim.x) {
+                float xv = __ldg(src + qq);
                 if (xv != xv) {
                     saw_nan = true;
                     xv = -INFINITY;
                 }
-                sh_logits[(q / N) * ldl + q % N] = xv;
+                sh_logits[(qq / N) * ldl + qq % N] = xv;
             }
         }
         __syncthreads();
-        if (per_thread) {
-            const int q = threadIdx.x;
-            if (q < nb) {
-                const float *l = sh_logits + (size_t)q * ldl;
-                switch (p.k) {
-                case 1: topk_thread<1>(p, b0 + q, l, sh_hist); break;
-                case 2: topk_thread<2>(p, b0 + q, l, sh_hist); break;
-                case 3: topk_thread<3>(p, b0 + q, l, sh_hist); break;
-                case 4: topk_thread<4>(p, b0 + q, l, sh_hist); break;
-                case 5: topk_thread<5>(p, b0 + q, l, sh_hist); break;
-                case 6: topk_thread<6>(p, b0 + q, l, sh_hist); break;
-                case 7: topk_thread<7>(p, b0 + q, l, sh_hist); break;
-                default: topk_thread<8>(p, b0 + q, l, sh_hist); break;
-                }
+        // threads beyond batch * grp (blockDim not a multiple) sit out whole warps
+        if ((int)(threadIdx.x & ~31u) < batch * grp) {
+            const bool active = q < nb;
+            const int t = b0 + q;
+            const float *l = sh_logits + (size_t)(active ? q : 0) * ldl;
+            int *kp = (keep && active) ? keep + (size_t)(t - t0) * p.k : nullptr;
+            switch (p.k) {
+            case 1: topk_group<1>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 2: topk_group<2>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 3: topk_group<3>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 4: topk_group<4>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 5: topk_group<5>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 6: topk_group<6>(p, t, l, s, grp, active, sh_hist, kp); break;
+            case 7: topk_group<7>(p, t, l, s, grp, active, sh_hist, kp); break;
+            default: topk_group<8>(p, t, l, s, grp, active, sh_hist, kp); break;
             }
-        } else {
-            for (int q = warp; q < nb; q += nw) topk_token(p, b0 + q, sh_logits + (size_t)q * ldl, sh_hist);
         }
     }
     __syncthreads();
@@ -331,64 +315,47 @@ __device__ __forceinline__ void decode_chunk(const uint32_t *__restrict__ packed
     reinterpret_cast<uint4 *>(wb)[q] = make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// Exclusive scan of src[0..n) into dst[0..n) by the whole block (warp
-// shuffles; `scratch` holds 72 ints); returns the sum.  src and dst may alias.
-__device__ int block_exclusive_scan(const int *src, int *dst, int n, int *scratch)
-{
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nw = blockDim.x >> 5;
-    int s = 0;
-    for (int e = lo; e < hi; ++e) s += src[e];
-    int incl = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
+// Shared-memory plan of the route kernel, in ints: the kept experts of the
+// block's rows, then either phase A (histogram + staged logits) or phases
+// B/C (offsets, bucket bases, partial sums), 16-byte aligned.
+struct RouteSmem {
+    int keep, a_hist, a_logits, off, cnt, red, total;
+    __host__ __device__ explicit RouteSmem(int N)
+    {
+        const int np4 = (N + 3) & ~3;
+        keep = 0;
+        a_hist = kSelCap;
+        a_logits = a_hist + np4;
+        const int a_end = a_logits + kLogitStageInts;
+        off = kSelCap;
+        cnt = off + N + 1;
+        red = cnt + N;
+        const int c_end = red + 2 * kRouteThreads;
+        total = a_end > c_end ? a_end : c_end;
     }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int w = lane < nw ? scratch[lane] : 0;
-        int wi = w;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, wi, off);
-            if (lane >= off) wi += o;
-        }
-        if (lane < nw) scratch[32 + lane] = wi - w;  // exclusive prefix of the warp totals
-        if (lane == nw - 1) scratch[64] = wi;         // block total
-    }
-    __syncthreads();
-    int run = scratch[32 + warp] + incl - s;
-    const int total = scratch[64];
-    for (int e = lo; e < hi; ++e) {
-        const int v = src[e];
-        dst[e] = run;
-        run += v;
-    }
-    __syncthreads();
-    return total;
-}
+};
 
 __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
 {
-    extern __shared__ int sh[];  // phase A: hist[N] + staged logits; phase C: off, tstart, cnt, scratch
+    extern __shared__ __align__(16) int sh[];
     const int N = p.N, k = p.k;
     const int nblk = gridDim.x;  // one histogram row per block
+    const RouteSmem lay(N);
 
     BFMOE_TRACE(0, threadIdx.x == 0, 0);
     pdl_trigger();  // the prep kernel may start now and run beside the routing
     // ---- phase A: top-k over this block's token range
-    float *sh_logits = reinterpret_cast<float *>(sh + ((N + 3) & ~3));
     bool saw_nan = false;
     const int tpb = (p.T + nblk - 1) / nblk;  // tokens per block
     const int t0 = min(p.T, (int)blockIdx.x * tpb), t1 = min(p.T, t0 + tpb);
-    topk_range(p, t0, t1, sh, sh_logits, saw_nan);
+    const bool kept = (t1 - t0) * k <= kSelCap;  // the scatter reads the experts from shared memory
+    int *keep = kept ? sh + lay.keep : nullptr;
+    int *hist_a = sh + lay.a_hist;
+    topk_range(p, t0, t1, hist_a, reinterpret_cast<float *>(sh + lay.a_logits), keep, saw_nan);
     const bool one_barrier = N <= kOneBarrierMaxN;  // one grid barrier
     const int np4 = (N + 3) & ~3;                    // histogram row stride, 16-byte multiple
-    for (int e = threadIdx.x; e < N; e += blockDim.x) p.hist[(size_t)blockIdx.x * (one_barrier ? np4 : N) + e] = sh[e];
+    for (int e = threadIdx.x; e < N; e += blockDim.x)
+        p.hist[(size_t)blockIdx.x * (one_barrier ? np4 : N) + e] = hist_a[e];
     if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     BFMOE_TRACE(0, threadIdx.x == 0, 1);
     const bool arrive = (int)blockIdx.x != p.skip_arrive_block;  // test hook: one block never arrives
@@ -401,37 +368,46 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     if (!grid_wait(p.sync, nblk, p.status)) return;
     BFMOE_TRACE(0, threadIdx.x == 0, 3);
 
-    int *off = sh;              // [N+1]
-    int *tstart = off + N + 1;  // [N+1]
-    int *cnt = tstart + N + 1;  // [N]
-    int *scratch = cnt + N;     // [72]
+    int *off = sh + lay.off;        // [N+1]
+    int *cnt = sh + lay.cnt;        // [N]
     if (one_barrier) {
         // ---- every block: expert totals and its own prefix over the blocks
-        // before it, from the expert-major histogram, staged in shared memory
-        // in chunks of experts with coalesced 16-byte loads
-        int *stage = sh + ((3 * N + 82 + 3) & ~3);  // [rb * np4], 16-byte aligned
-        const int rb = max(1, kHistStageInts / np4);  // histogram rows per chunk
-        for (int e = threadIdx.x; e < N; e += blockDim.x) {
-            off[e] = 0;
-            cnt[e] = 0;
-        }
-        for (int b0 = 0; b0 < nblk; b0 += rb) {
-            const int nb = min(rb, nblk - b0);
-            copy_g2s(reinterpret_cast<const int4 *>(p.hist + (size_t)b0 * np4), reinterpret_cast<int4 *>(stage),
-                     nb * np4 / 4, threadIdx.x, blockDim.x);
-            __syncthreads();
-            for (int e = threadIdx.x; e < N; e += blockDim.x) {
-                int tot = 0, pre = 0;
-                for (int b = 0; b < nb; ++b) {
-                    const int v = stage[b * np4 + e];
-                    tot += v;
-                    pre += (b0 + b < (int)blockIdx.x) ? v : 0;
+        // before it, straight from the block-major histogram: `parts`
+        // threads per expert take every parts-th row (a warp reads 32
+        // consecutive experts of a row), 32 loads in flight per thread
+        int *red = sh + lay.red;  // [2][parts * N]
+        const int parts = max(1, (int)blockDim.x / N);
+        for (int idx = threadIdx.x; idx < parts * N; idx += blockDim.x) {
+            const int e = idx % N, part = idx / N;
+            int tot = 0, pre = 0;
+            for (int b0 = part; b0 < nblk; b0 += 32 * parts) {
+                int v[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int b = b0 + u * parts;
+                    v[u] = b < nblk ? __ldcg(p.hist + (size_t)b * np4 + e) : 0;
                 }
-                off[e] += tot;
-                cnt[e] += pre;  // becomes the block's bucket base below
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    tot += v[u];
+                    pre += (b0 + u * parts < (int)blockIdx.x) ? v[u] : 0;
+                }
             }
-            __syncthreads();
+            red[idx] = tot;
+            red[parts * N + idx] = pre;
         }
+        __syncthreads();
+        BFMOE_TRACE(0, threadIdx.x == 0, 6);
+        for (int e = threadIdx.x; e < N; e += blockDim.x) {
+            int tot = 0, pre = 0;
+            for (int q = 0; q < parts; ++q) {
+                tot += red[q * N + e];
+                pre += red[parts * N + q * N + e];
+            }
+            off[e] = tot;  // scanned into bucket offsets below
+            cnt[e] = pre;  // becomes the block's bucket base below
+        }
+        __syncthreads();
     } else {
         // ---- phase B: one warp per expert, exclusive prefix over the blocks
         const int warp = (int)(gtid >> 5), lane = threadIdx.x & 31;
@@ -470,38 +446,42 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     }
     BFMOE_TRACE(0, threadIdx.x == 0, 4);
 
-    // ---- phase C: bucket offsets, tile list, ranks and scatter
-    for (int e = threadIdx.x; e < N; e += blockDim.x)
-        tstart[e] = p.tile_rows > 0 ? (off[e] + p.tile_rows - 1) / p.tile_rows : 0;
-    __syncthreads();
-    const int rsum = block_exclusive_scan(off, off, N, scratch);
-    const int ntiles = p.in_tiles ? block_exclusive_scan(tstart, tstart, N, scratch) : 0;
-    if (threadIdx.x == 0) {
-        off[N] = rsum;
-        tstart[N] = ntiles;
-    }
-    for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] += off[e];
-    __syncthreads();
-    if (blockIdx.x == 0) {
-        for (int e = threadIdx.x; e <= N; e += blockDim.x) p.offsets[e] = off[e];
-        if (threadIdx.x == 0 && p.n_in_tiles) *p.n_in_tiles = ntiles;
-    }
-    if (p.in_tiles) {
-        for (int e = (int)gtid; e < N; e += (int)gthreads) {
-            const int n_e = off[e + 1] - off[e];
-            int q = tstart[e];
-            for (int r = 0; r < n_e; r += p.tile_rows, ++q)
-                p.in_tiles[q] = make_int4(e, off[e] + r, min(p.tile_rows, n_e - r), 0);
-        }
-    }
+    // ---- phase C: bucket offsets and bucket bases by one warp (lane-serial
+    // chunks + a shuffle scan), then ranks and scatter
     if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (N + 31) / 32;
+        const int lo = min(N, lane * per), hi = min(N, lo + per);
+        int srow = 0;
+        for (int e = lo; e < hi; ++e) srow += off[e];
+        int irow = srow;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, irow, o);
+            if (lane >= o) irow += a;
+        }
+        int run = irow - srow;
+        for (int e = lo; e < hi; ++e) {
+            const int n = off[e];
+            off[e] = run;
+            cnt[e] += run;
+            run += n;
+        }
+        if (lane == 31) off[N] = irow;
+    }
+    __syncthreads();
+    BFMOE_TRACE(0, threadIdx.x == 0, 8);
+    if (blockIdx.x == 0)
+        for (int e = threadIdx.x; e <= N; e += blockDim.x) p.offsets[e] = off[e];
+    if (threadIdx.x < 32) {
+        // one warp ranks the block's rows in row order: stable inside buckets
         const int lane = threadIdx.x;
         const unsigned lt = (1u << lane) - 1u;
         const int i0 = t0 * k, i1 = t1 * k;
         for (int c0 = i0; c0 < i1; c0 += 32) {
             const int i = c0 + lane;
             const bool valid = i < i1;
-            const int e = valid ? p.topk_idx[i] : -1;
+            const int e = valid ? (kept ? keep[i - i0] : p.topk_idx[i]) : -1;
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             const int pos = valid ? cnt[e] + __popc(peers & lt) : 0;
             __syncwarp();
@@ -510,18 +490,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             if (valid) {
                 p.perm[pos] = i;
                 if (p.row_pos) p.row_pos[i] = pos;
+                if (p.row_tok) {
+                    p.row_tok[pos] = i / k;
+                    p.row_exp[pos] = e;
+                }
             }
         }
     }
     BFMOE_TRACE(0, threadIdx.x == 0, 5);
 }
 
-__host__ inline size_t route_smem_bytes(int N)
-{
-    const size_t ldl = N <= kThreadTopkMaxN ? N + 1 : N;
-    const size_t a = (size_t)((N + 3) & ~3) * 4 + (size_t)route_batch_tokens(N) * ldl * 4;  // phase A
-    const size_t c = (size_t)(((3 * N + 82 + 3) & ~3) + kHistStageInts) * 4;               // phase B/C
-    return a > c ? a : c;
-}
+__host__ inline size_t route_smem_bytes(int N) { return (size_t)RouteSmem(N).total * 4; }
 
 }  // namespace bfmoe
