@@ -368,7 +368,7 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     const size_t c_smem = contract_smem_bytes(d);
     auto kc = BN == 256 ? k_contract<256> : (BN == 128 ? k_contract<128> : k_contract<64>);
     if (!ensure_smem((const void *)kc, c_smem)) return BFMOE_ERR_CUDA;
-    if (launch(kc, dim3(std::min(nunits, sms)), dim3(kContractThreads), c_smem, st, true, false, cpar) !=
+    if (launch(kc, dim3(std::min(nunits, sms)), dim3(contract_threads(BN)), c_smem, st, true, false, cpar) !=
         cudaSuccess)
         return BFMOE_ERR_CUDA;
     mark(rec, st);

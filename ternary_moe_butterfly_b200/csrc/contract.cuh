@@ -32,7 +32,11 @@
 
 namespace bfmoe {
 
-constexpr int kContractThreads = 320;  // 2 control warps + 8 epilogue warps
+// Epilogue warps per TMEM lane quadrant (each takes 1/parts of a row's
+// columns), and the CTA size: a producer warp, an MMA warp, 4 * parts
+// epilogue warps.
+__host__ __device__ constexpr int epi_parts(int) { return 2; }
+__host__ __device__ constexpr int contract_threads(int BN) { return 64 + 128 * epi_parts(BN); }
 constexpr int kStages = 3;
 
 
@@ -151,10 +155,10 @@ __device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred)
 // Output-butterfly stages 0 .. log2(BN)-1 of one row held in TMEM columns
 // [tbase, tbase + BN) of this warp's lanes, then store to `out` (if
 // non-null).  `tab` is the row's expert's slice table in the output-table
-// order (shared or global memory, as the caller's pointer type says).  Two
-// warps share the row's lanes: `part` (0 or 1) selects which half of the
-// 32-column blocks (pass 1) and of the 8-column groups (pass 2) this warp
-// takes; `bar_id` is a 64-thread named barrier for the pair.
+// order (shared or global memory, as the caller's pointer type says).
+// epi_parts(BN) warps share the row's lanes: `part` selects this warp's share
+// of the 32-column blocks (pass 1) and of the 8-column groups (pass 2);
+// `bar_id` is the named barrier of those warps.
 template <int BN, typename Tab>
 __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__restrict__ out, float scale,
                                              int part, int bar_id)
@@ -164,6 +168,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
     constexpr int M2 = 1 << G2;
     constexpr int NB = BN / 32;
     constexpr int PER2 = G2 * 8 * (M2 / 2);
+    constexpr int PARTS = epi_parts(BN);
     // pass 1: stages 0..4 inside each 32-column block; the next block's TMEM
     // load is in flight while this one rotates
     auto pass1_block = [&](int blk, float (&v)[32]) {
@@ -191,7 +196,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
         tmem_st32(tbase + (uint32_t)(blk * 32), v);
     };
     {
-        constexpr int NBH = NB / 2;  // blocks per warp
+        constexpr int NBH = NB / PARTS;  // blocks per warp
         const int b0 = part * NBH;
         float va[32], vb[32];
         tmem_ld32_async(tbase + (uint32_t)(b0 * 32), va);
@@ -210,11 +215,12 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
     }
     tmem_st_wait();
     BFMOE_TRACE(2, threadIdx.x == 64, 9);
-    named_bar_sync(bar_id, 64);
+    named_bar_sync(bar_id, 32 * PARTS);
     BFMOE_TRACE(2, threadIdx.x == 64, 10);
     // pass 2: stages 5..SIN-1 on columns c0 + q + 32 m, 8-column groups
+    constexpr int GPP = 4 / PARTS;  // groups per warp
 #pragma unroll 1
-    for (int grp = part * 2; grp < part * 2 + 2; ++grp) {
+    for (int grp = part * GPP; grp < (part + 1) * GPP; ++grp) {
         const int c0 = grp * 8;
         float v[8][M2];
 #pragma unroll
@@ -278,8 +284,9 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams p)
+__global__ void __launch_bounds__(contract_threads(BN), 1) k_contract(ContractParams p)
 {
+    constexpr int PARTS = epi_parts(BN);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int d = p.d;
     const int KC = d / kBK;
@@ -307,7 +314,7 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);
+            mbar_init(&tempty[b], 4 * PARTS);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -390,8 +397,8 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             if (!mbar_wait(drain, 0)) set_status(p.status, BFMOE_ERR_TIMEOUT);
         }
     } else {
-        // epilogue warps 2..9: warp w owns TMEM lanes 32*(w % 4) .. +31 and
-        // half of the row's columns (part = (w - 2) / 4)
+        // epilogue warps 2..: warp w owns TMEM lanes 32*(w % 4) .. +31 and
+        // 1/PARTS of the row's columns (part = (w - 2) / 4)
         const int lane_base = (warp & 3) * 32;
         const int part = (warp - 2) >> 2;
         const int bar_id = 1 + (warp & 3);
@@ -413,7 +420,7 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
             // the rows are in bucket order: stage the slice tables of the
             // first and last row's experts while the MMA runs
             const int ea = __shfl_sync(0xffffffffu, e, 0), eb = __shfl_sync(0xffffffffu, e, 31);
-            named_bar_sync(bar_id, 64);  // the pair is done with the previous unit's tables
+            named_bar_sync(bar_id, 32 * PARTS);  // the quadrant's warps are done with the previous tables
             {
                 // the two experts' slice tables: contiguous copies
                 constexpr int SL4 = SIN * HB / 2;  // float4 per slice table
@@ -421,14 +428,14 @@ __global__ void __launch_bounds__(kContractThreads, 1) k_contract(ContractParams
                 for (int t = 0; t < 2; ++t)
                     copy_g2s(reinterpret_cast<const float4 *>(p.coef_p + (size_t)(t ? eb : ea) * p.L * half +
                                                               (size_t)nh * SIN * HB),
-                             reinterpret_cast<float4 *>(ptab + (size_t)t * SIN * HB), SL4, pt, 64);
+                             reinterpret_cast<float4 *>(ptab + (size_t)t * SIN * HB), SL4, pt, 32 * PARTS);
             }
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 13);
             bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
             // both warps sharing these lanes take the same branch (they meet
             // at named barriers inside epilogue_row); the barrier also makes
             // the staged tables visible to the pair
-            ok = bar_red_and(bar_id, 64, ok);
+            ok = bar_red_and(bar_id, 32 * PARTS, ok);
             if (!ok) {
                 if (lane == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
                 break;
