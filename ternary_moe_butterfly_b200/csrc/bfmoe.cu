@@ -309,6 +309,8 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     pp.packed = reinterpret_cast<const uint32_t *>(packed);
     pp.wdec = wdec;
     pp.status = status;
+    pp.x = x;
+    pp.x_bytes = (size_t)T_ * d * sizeof(T);
     // one block per SM: the prep shares the SMs with the routing, whose
     // latency chain must keep most of the issue slots
     const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, sms));

@@ -25,6 +25,8 @@ struct PrepParams {
     const uint32_t *packed;    // packed base (header + words)
     __half *wdec;              // decoded base, GEMM B-operand blocks
     uint32_t *status;
+    const void *x;             // layer input, prefetched into L2 ([x_bytes], 16-byte multiple)
+    size_t x_bytes;
 };
 
 // {cos, sin} tables of every expert in consumption order: theta -> the
@@ -42,6 +44,22 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
     // this grid (and so for the routing) to complete before reading anything
     BFMOE_TRACE(4, threadIdx.x == 0, 0);
     pdl_trigger();
+    if (threadIdx.x == 0 && p.x) {
+        // the input-butterfly kernel gathers x right after the routing: bring
+        // this block's share of it into L2 now (off the routing's path)
+        const size_t share = ((p.x_bytes + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
+        const size_t lo = (size_t)blockIdx.x * share;
+        if (lo < p.x_bytes) {
+            const size_t n = p.x_bytes - lo < share ? p.x_bytes - lo : share;
+            for (size_t o = 0; o < n; o += (1u << 20)) {
+                const uint32_t c = (uint32_t)(n - o < (1u << 20) ? n - o : (1u << 20));
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                                 reinterpret_cast<const char *>(p.x) + lo + o),
+                             "r"(c)
+                             : "memory");
+            }
+        }
+    }
     constexpr int L = LL, d = 1 << LL, half = d >> 1;
     constexpr int tab = L * half;
     const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
