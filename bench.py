@@ -359,7 +359,7 @@ def run_ours(args, w):
     models = {
         "contract": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
         "expert_in": ("alu", 4.0 * rot, "Tops/s"),
-        "combine": ("hbm", R * d * 4 + T * d * xb + T * k * 8, "GB/s"),
+        "combine": ("hbm", R * d * 2 + T * d * xb + R * 4, "GB/s"),
         "route": ("hbm", T * N * 4 + T * k * 12, "GB/s"),
     }
     dom = max(prof, key=prof.get) if prof else None
