@@ -43,8 +43,15 @@
  * return an error code at once.  Errors that only the device can see (NaN
  * logits, fp16 overflow of a rotated row, a malformed packed base, a wait
  * that timed out) are written to a status word at the start of the
- * workspace; read it with bfmoe_sync_status.  A failed kernel launch returns
- * BFMOE_ERR_CUDA.
+ * workspace; read it with bfmoe_sync_status.  Each call clears the status
+ * word when it starts.  A failed kernel launch returns BFMOE_ERR_CUDA.
+ *
+ * Workspaces: the first 32 bytes hold the status word and the routing's
+ * grid-barrier words.  Their content on a workspace's first use does not
+ * matter (the routing clears them on a launch it has not seen), and every
+ * call leaves them ready for the next one, so no call clears them with a
+ * separate copy.  Calls that share a workspace must be ordered (one stream,
+ * or events).
  *
  * Limits: d is a power of two in [64, 4096]; 1 <= N <= 4096;
  * 1 <= k <= min(N, 8); 1 <= T <= 2^24 / k; x and y are fp32 or bf16,

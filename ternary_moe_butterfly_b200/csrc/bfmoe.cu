@@ -3,8 +3,10 @@
 // every entry point are in include/bfmoe.h.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 #include <map>
+#include <random>
 #include <mutex>
 #include <utility>
 
@@ -95,7 +97,7 @@ FwdLayout fwd_layout(int T, int d, int N, int k)
         o += align_up(bytes);
         return at;
     };
-    l.status = take(16);
+    l.status = take(32);
     l.topk_idx = take(R * 4);
     l.gates = take(R * 4);
     l.perm = take(R * 4);
@@ -193,6 +195,31 @@ void *static_scratch()
 // first grid barrier, or -1.
 int g_skip_arrive_block = -1;
 
+// Launch tokens of the routing barrier: unique per launch within the process,
+// from a random 64-bit start (a fresh workspace's epoch word matches one only
+// by a 2^-64 chance).
+std::atomic<unsigned long long> g_token{0};
+unsigned long long next_token()
+{
+    static const unsigned long long base = [] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32) ^ (unsigned long long)rd() ^ 0x9e3779b97f4a7c15ull;
+    }();
+    return base + 2ull * g_token.fetch_add(1, std::memory_order_relaxed) + 1ull;
+}
+
+// The status / barrier header at the start of every workspace (32 bytes):
+// status word, barrier counter, departed counter, pad, 64-bit epoch.
+void set_header(RouteParams &rp, uint8_t *hdr)
+{
+    uint32_t *w = reinterpret_cast<uint32_t *>(hdr);
+    rp.status = w;
+    rp.sync = w + 1;
+    rp.departed = w + 2;
+    rp.epoch = reinterpret_cast<unsigned long long *>(hdr + 16);
+    rp.token = next_token();
+}
+
 // Optional per-kernel event recorder used by bfmoe_forward_profile.
 struct StageRec {
     cudaEvent_t ev[BFMOE_MAX_STAGES + 1];
@@ -234,7 +261,10 @@ cudaError_t launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// The routing kernel, launched cooperatively on as many blocks as fit.
+// The routing kernel, launched cooperatively on as many blocks as fit, with a
+// programmatic dependency on whatever precedes it on the stream: it becomes
+// resident while the previous call's last kernel runs and waits for it
+// before touching memory.
 bfmoe_status launch_route(RouteParams rp, cudaStream_t st)
 {
     const size_t smem = route_smem_bytes(rp.N);
@@ -248,7 +278,7 @@ bfmoe_status launch_route(RouteParams rp, cudaStream_t st)
     const int by_tokens = (int)std::min<long long>(kMaxRouteBlocks, ((long long)rp.T + 31) / 32);
     const int grid = std::max(1, std::min(std::min(std::min(sms, occ * sms), kMaxRouteBlocks), by_tokens));
     rp.skip_arrive_block = g_skip_arrive_block;
-    if (launch(k_route, dim3(grid), dim3(kRouteThreads), smem, st, false, true, rp) != cudaSuccess)
+    if (launch(k_route, dim3(grid), dim3(kRouteThreads), smem, st, true, true, rp) != cudaSuccess)
         return BFMOE_ERR_CUDA;
     return BFMOE_OK;
 }
@@ -274,7 +304,6 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     const int sms = device_sms();
     if (sms <= 0) return BFMOE_ERR_CUDA;
 
-    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
     mark(rec, st);
 
     RouteParams rp{};
@@ -289,8 +318,7 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     rp.offsets = reinterpret_cast<int32_t *>(ws + l.offsets);
     rp.hist = reinterpret_cast<int32_t *>(ws + l.hist);
     rp.total = reinterpret_cast<int32_t *>(ws + l.total);
-    rp.sync = status + 1;
-    rp.status = status;
+    set_header(rp, ws + l.status);
     rp.row_tok = row_tok;
     rp.row_exp = row_exp;
     rp.d = d;
@@ -491,8 +519,6 @@ bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk
     if (ws_bytes < l.total_bytes) return BFMOE_ERR_WORKSPACE;
     uint8_t *w = reinterpret_cast<uint8_t *>(ws);
     cudaStream_t st = as_stream(stream);
-    uint32_t *status = reinterpret_cast<uint32_t *>(w + l.status);
-    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
     RouteParams rp{};
     rp.logits = logits;
     rp.T = T;
@@ -504,8 +530,7 @@ bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk
     rp.offsets = offsets;
     rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
     rp.total = reinterpret_cast<int32_t *>(w + l.total);
-    rp.sync = status + 1;
-    rp.status = status;
+    set_header(rp, w + l.status);
     s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
     return launched();
@@ -525,8 +550,6 @@ bfmoe_status bfmoe_route_static(const float *logits, int T, int N, int k, int32_
     uint8_t *w = reinterpret_cast<uint8_t *>(static_scratch());
     if (!w) return BFMOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
-    uint32_t *status = reinterpret_cast<uint32_t *>(w + l.status);
-    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return BFMOE_ERR_CUDA;
     RouteParams rp{};
     rp.logits = logits;
     rp.T = T;
@@ -538,8 +561,7 @@ bfmoe_status bfmoe_route_static(const float *logits, int T, int N, int k, int32_
     rp.offsets = offsets;
     rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
     rp.total = reinterpret_cast<int32_t *>(w + l.total);
-    rp.sync = status + 1;
-    rp.status = status;
+    set_header(rp, w + l.status);
     s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
     return launched();

@@ -53,7 +53,10 @@ struct RouteParams {
     int32_t *offsets;    // [N+1]
     int32_t *hist;       // [gridDim][N] -> per-block bucket bases
     int32_t *total;      // [N]
-    uint32_t *sync;      // grid barrier counter, zero at launch
+    uint32_t *sync;      // grid barrier counter (returned to zero by the last block to leave)
+    uint32_t *departed;  // blocks done with the barrier counter
+    unsigned long long *epoch;  // launch token of the last reset of the counters
+    unsigned long long token;   // this launch's token
     uint32_t *status;
     int skip_arrive_block;  // test hook: this block never reaches barrier 1 (-1: none)
     int d;
@@ -84,6 +87,60 @@ __host__ __device__ inline int route_batch_tokens(int N)
 __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b)
 {
     return va > vb || (va == vb && a < b);
+}
+
+// The barrier counters live in the caller's workspace and need no clearing
+// between calls: the last block to leave a launch returns them to zero, and a
+// launch whose token differs from the stored epoch (a fresh workspace, whose
+// words may hold anything) has block 0 clear them and publish the token
+// before any block arrives.
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Block 0, thread 0, first thing: clear the counters if this launch's token
+// is new to the workspace.
+__device__ __forceinline__ void grid_epoch_open(uint32_t *ctr, uint32_t *departed, unsigned long long *epoch,
+                                                unsigned long long token)
+{
+    if (ld_acquire_u64(epoch) != token) {
+        atomicExch(ctr, 0u);
+        atomicExch(departed, 0u);
+        __threadfence();
+        st_release_u64(epoch, token);
+    }
+}
+
+// Thread 0 of every block, before arriving: wait (bounded) until the
+// counters are known clear for this launch.
+__device__ __forceinline__ bool grid_epoch_wait(const unsigned long long *epoch, unsigned long long token)
+{
+    if (ld_acquire_u64(epoch) == token) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_u64(epoch) != token)
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+// Every block, once, after its last use of the counter (also on a timeout):
+// the last one returns the counters to zero for the next launch.
+__device__ __forceinline__ void grid_depart(uint32_t *ctr, uint32_t *departed, int nblk)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(departed, 1u) == (uint32_t)nblk - 1u) {
+            atomicExch(ctr, 0u);
+            atomicExch(departed, 0u);
+        }
+    }
 }
 
 // Split-phase grid-wide barrier on a monotonically increasing counter:
@@ -343,7 +400,14 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     const RouteSmem lay(N);
 
     BFMOE_TRACE(0, threadIdx.x == 0, 0);
+    pdl_wait();     // (launched after the previous call's kernels: they read this workspace)
     pdl_trigger();  // the prep kernel may start now and run beside the routing
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        // a new call's status; every other status write of this launch comes
+        // after the grid barrier, which block 0 reaches after this store
+        *reinterpret_cast<volatile uint32_t *>(p.status) = 0u;
+        grid_epoch_open(p.sync, p.departed, p.epoch, p.token);
+    }
     // ---- phase A: top-k over this block's token range
     bool saw_nan = false;
     const int tpb = (p.T + nblk - 1) / nblk;  // tokens per block
@@ -356,16 +420,35 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     const int np4 = (N + 3) & ~3;                    // histogram row stride, 16-byte multiple
     for (int e = threadIdx.x; e < N; e += blockDim.x)
         p.hist[(size_t)blockIdx.x * (one_barrier ? np4 : N) + e] = hist_a[e];
-    if (__any_sync(0xffffffffu, saw_nan) && (threadIdx.x & 31) == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
+    const bool nan_here = __syncthreads_or(saw_nan);
     BFMOE_TRACE(0, threadIdx.x == 0, 1);
     const bool arrive = (int)blockIdx.x != p.skip_arrive_block;  // test hook: one block never arrives
+    {
+        __shared__ int epoch_ok;
+        if (threadIdx.x == 0) epoch_ok = grid_epoch_wait(p.epoch, p.token) ? 1 : 0;
+        __syncthreads();
+        if (!epoch_ok) {
+            if (threadIdx.x == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
+            grid_depart(p.sync, p.departed, nblk);
+            return;
+        }
+    }
     if (arrive) grid_arrive(p.sync);
 
     const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t gthreads = (size_t)gridDim.x * blockDim.x;
     BFMOE_TRACE(0, threadIdx.x == 0, 2);
-    if (!arrive) return;
-    if (!grid_wait(p.sync, nblk, p.status)) return;
+    if (!arrive) {
+        grid_depart(p.sync, p.departed, nblk);
+        return;
+    }
+    const bool one_ok = grid_wait(p.sync, nblk, p.status);
+    if (one_ok && one_barrier) grid_depart(p.sync, p.departed, nblk);  // the only barrier is behind us
+    if (!one_ok) {
+        grid_depart(p.sync, p.departed, nblk);
+        return;
+    }
+    if (nan_here && threadIdx.x == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     BFMOE_TRACE(0, threadIdx.x == 0, 3);
 
     int *off = sh + lay.off;        // [N+1]
@@ -437,7 +520,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
             if (lane == 0) p.total[e] = running;
         }
         grid_arrive(p.sync);
-        if (!grid_wait(p.sync, 2 * nblk, p.status)) return;
+        const bool two_ok = grid_wait(p.sync, 2 * nblk, p.status);
+        grid_depart(p.sync, p.departed, nblk);
+        if (!two_ok) return;
         for (int e = threadIdx.x; e < N; e += blockDim.x) {
             off[e] = p.total[e];
             cnt[e] = p.hist[(size_t)blockIdx.x * N + e];

@@ -262,6 +262,36 @@ def test_forward_twice_same_workspace_is_deterministic(bf):
     assert torch.equal(y1, y2)
 
 
+def test_forward_workspace_header_garbage_and_graph_replay(bf):
+    # the status / barrier words of a fresh workspace may hold anything, and
+    # a graph replays the same launch (same barrier token) back to back
+    inp = wl.make_inputs("headline", T=300)
+    x = to_x(inp)
+    packed = bf.pack_base(dev(inp.w_base), inp.alpha)
+    lg, th, ph = dev(inp.logits), dev(inp.theta), dev(inp.phi)
+    ref, ws0 = bf.forward(x, lg, 2, packed, th, ph)
+    assert bf.sync_status(ws0) == bf.OK
+    ws = torch.full_like(ws0, 0xA5)
+    y, _ = bf.forward(x, lg, 2, packed, th, ph, ws=ws)
+    assert bf.sync_status(ws) == bf.OK
+    assert torch.equal(y, ref)
+    stream = torch.cuda.Stream()
+    out = torch.empty_like(ref)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        bf.forward(x, lg, 2, packed, th, ph, ws=ws, out=out, stream=stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            bf.forward(x, lg, 2, packed, th, ph, ws=ws, out=out, stream=stream)
+        for _ in range(3):
+            out.zero_()
+            g.replay()
+            stream.synchronize()
+            assert torch.equal(out, ref)
+    assert bf.sync_status(ws) == bf.OK
+    del g
+
+
 # ------------------------------------------------------ failure detection
 # A routing block that never reaches the grid barrier (host-side test hook)
 # makes the others' bounded waits run out: the call must report
@@ -279,16 +309,28 @@ def test_route_barrier_timeout_reports_status(bf):
         bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, -1)
     assert st == bf.ERR_TIMEOUT
     check_route(bf, lg, k)
+    # the barrier words left by the timed-out call are usable again
+    idx, gates, perm, offsets, _ = bf.route(dev(lg), k, ws=ws)
+    assert bf.sync_status(ws) == bf.OK
+    ref = oracle.route(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ref[0])
+    assert np.array_equal(perm.cpu().numpy(), ref[2])
 
 
 def test_forward_barrier_timeout_reports_status(bf):
     inp = wl.make_inputs("headline", T=300)
     bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, 1)
     try:
-        _, _, st = run_forward(bf, inp)
+        _, ws_timed_out, st = run_forward(bf, inp)
     finally:
         bf.bfmoe_debug_set(bf.DEBUG_SKIP_ARRIVE_BLOCK, -1)
     assert st == bf.ERR_TIMEOUT
     y, ws, st = run_forward(bf, inp)
     assert st == bf.OK
-    check_close(y.float().cpu().numpy(), oracle_forward(inp), "after timeout")
+    ref = oracle_forward(inp)
+    check_close(y.float().cpu().numpy(), ref, "after timeout")
+    # the same workspace, whose barrier words the timed-out call left behind
+    y2, _ = bf.forward(to_x(inp), dev(inp.logits), inp.wl.k, bf.pack_base(dev(inp.w_base), inp.alpha),
+                       dev(inp.theta), dev(inp.phi), ws=ws_timed_out)
+    assert bf.sync_status(ws_timed_out) == bf.OK
+    check_close(y2.float().cpu().numpy(), ref, "same workspace after timeout")
