@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
 
     BFMOE_TRACE(0, threadIdx.x == 0, 0);
     pdl_wait();     // (launched after the previous call's kernels: they read this workspace)
-    pdl_trigger();  // the prep kernel may start now and run beside the routing
+    BFMOE_TRACE(0, threadIdx.x == 0, 11);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         // a new call's status; every other status write of this launch comes
         // after the grid barrier, which block 0 reaches after this store
@@ -448,6 +448,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         grid_depart(p.sync, p.departed, nblk);
         return;
     }
+    // the prep kernel may start now and run beside the rest of the routing
+    // (earlier, it slows the top-k and the barrier more than it gains)
+    pdl_trigger();
     if (nan_here && threadIdx.x == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     BFMOE_TRACE(0, threadIdx.x == 0, 3);
 
