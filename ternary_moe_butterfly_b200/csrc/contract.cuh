@@ -40,9 +40,11 @@ __host__ __device__ constexpr int contract_threads(int BN) { return 64 + 128 * e
 constexpr int kStages = 3;
 
 
-// Shared-memory cos/sin tables staged per pair of epilogue warps: two
-// experts x slice_stages(BN) stages x BN/2 pairs.
-__host__ __device__ constexpr int pair_table_floats2(int BN) { return 2 * slice_stages(BN) * (BN / 2); }
+// Shared-memory cos/sin tables staged per TMEM lane quadrant: two experts x
+// slice_stages(BN) stages x BN/2 pairs, the second table 16 bytes further on
+// so that a warp whose rows use both tables reads them from distinct banks.
+__host__ __device__ constexpr int staged_slice_stride(int BN) { return slice_stages(BN) * (BN / 2) + 2; }
+__host__ __device__ constexpr int pair_table_floats2(int BN) { return 2 * staged_slice_stride(BN); }
 
 // Output tables hold each expert's {cos a, sin a} of phi in the order the
 // epilogue and the combine consume them.  For each BN-column slice nh:
@@ -222,56 +224,62 @@ __device__ __forceinline__ void epilogue_row(uint32_t tbase, Tab tab, __half *__
 #pragma unroll 1
     for (int grp = part * GPP; grp < (part + 1) * GPP; ++grp) {
         const int c0 = grp * 8;
-        float v[8][M2];
-#pragma unroll
-        for (int m = 0; m < M2; ++m) {
-            tmem_ld4_nowait(tbase + (uint32_t)(c0 + 32 * m), v[0][m], v[1][m], v[2][m], v[3][m]);
-            tmem_ld4_nowait(tbase + (uint32_t)(c0 + 4 + 32 * m), v[4][m], v[5][m], v[6][m], v[7][m]);
-        }
-        tmem_ld_wait();
         const Tab t2 = tab + (NB * 80 + grp * PER2);
+        // the group's 8 columns in two halves of 4 (fewer live registers);
+        // the fp16 results of both halves meet in h for the 32-byte stores
+        uint32_t h[M2 * 4];
 #pragma unroll
-        for (int ls = 0; ls < G2; ++ls) {
-            const int h = 1 << ls;
+        for (int qh = 0; qh < 8; qh += 4) {
+            float v[4][M2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                if constexpr (M2 >= 4) {
-                    // rotations ri, ri+1 of column q: one paired table load
+            for (int m = 0; m < M2; ++m)
+                tmem_ld4_nowait(tbase + (uint32_t)(c0 + qh + 32 * m), v[0][m], v[1][m], v[2][m], v[3][m]);
+            tmem_ld_wait();
 #pragma unroll
-                    for (int ri = 0; ri < M2 / 2; ri += 2) {
-                        const float4 w = t2.ld4((ls * 8 + q) * (M2 / 2) + ri);
-                        const int m0 = insert_zero_bit(ri, ls), m1 = insert_zero_bit(ri + 1, ls);
-                        if (ls > 0) {
-                            float2 a = make_float2(v[q][m0], v[q][m1]), b = make_float2(v[q][m0 + h], v[q][m1 + h]);
-                            rot2(a, b, make_float2(w.x, w.y), make_float2(w.z, w.w));
-                            v[q][m0] = a.x;
-                            v[q][m1] = a.y;
-                            v[q][m0 + h] = b.x;
-                            v[q][m1 + h] = b.y;
-                        } else {
-                            rot1(v[q][m0], v[q][m0 + h], w.x, w.z);
-                            rot1(v[q][m1], v[q][m1 + h], w.y, w.w);
+            for (int ls = 0; ls < G2; ++ls) {
+                const int hs = 1 << ls;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q = qh + qq;
+                    if constexpr (M2 >= 4) {
+                        // rotations ri, ri+1 of column q: one paired table load
+#pragma unroll
+                        for (int ri = 0; ri < M2 / 2; ri += 2) {
+                            const float4 w = t2.ld4((ls * 8 + q) * (M2 / 2) + ri);
+                            const int m0 = insert_zero_bit(ri, ls), m1 = insert_zero_bit(ri + 1, ls);
+                            if (ls > 0) {
+                                float2 a = make_float2(v[qq][m0], v[qq][m1]);
+                                float2 b = make_float2(v[qq][m0 + hs], v[qq][m1 + hs]);
+                                rot2(a, b, make_float2(w.x, w.y), make_float2(w.z, w.w));
+                                v[qq][m0] = a.x;
+                                v[qq][m1] = a.y;
+                                v[qq][m0 + hs] = b.x;
+                                v[qq][m1 + hs] = b.y;
+                            } else {
+                                rot1(v[qq][m0], v[qq][m0 + hs], w.x, w.z);
+                                rot1(v[qq][m1], v[qq][m1 + hs], w.y, w.w);
+                            }
                         }
+                    } else {
+                        // one rotation per column and stage: the pair partner
+                        // is the next column's
+                        const float2 cs = t2.cs((ls * 8 + q) * (M2 / 2));
+                        rot1(v[qq][0], v[qq][hs], cs.x, cs.y);
                     }
-                } else {
-                    // one rotation per column and stage: the pair partner is
-                    // the next column's
-                    const float2 cs = t2.cs((ls * 8 + q) * (M2 / 2));
-                    rot1(v[q][0], v[q][h], cs.x, cs.y);
                 }
             }
-        }
-        if (out) {
-            // alpha * gate, fp16, the group's M2 x 8 values as one contiguous run
-            // (slot row layout [group][m][q], described with CombineParams); 32-byte stores
-            uint32_t h[M2 * 4];
+            // alpha * gate, fp16, packed in [m][q] order
 #pragma unroll
             for (int m = 0; m < M2; ++m)
 #pragma unroll
-                for (int q = 0; q < 8; q += 2) {
-                    __half2 hv = __floats2half2_rn(scale * v[q][m], scale * v[q + 1][m]);
-                    h[m * 4 + q / 2] = *reinterpret_cast<uint32_t *>(&hv);
+                for (int qq = 0; qq < 4; qq += 2) {
+                    __half2 hv = __floats2half2_rn(scale * v[qq][m], scale * v[qq + 1][m]);
+                    h[m * 4 + (qh + qq) / 2] = *reinterpret_cast<uint32_t *>(&hv);
                 }
+        }
+        if (out) {
+            // the group's M2 x 8 values as one contiguous run (slot row
+            // layout [group][m][q], described with CombineParams)
             __half *dst = out + grp * (8 * M2);
 #pragma unroll
             for (int w = 0; w < M2 / 2; ++w)
@@ -428,7 +436,8 @@ __global__ void __launch_bounds__(contract_threads(BN), 1) k_contract(ContractPa
                 for (int t = 0; t < 2; ++t)
                     copy_g2s(reinterpret_cast<const float4 *>(p.coef_p + (size_t)(t ? eb : ea) * p.L * half +
                                                               (size_t)nh * SIN * HB),
-                             reinterpret_cast<float4 *>(ptab + (size_t)t * SIN * HB), SL4, pt, 32 * PARTS);
+                             reinterpret_cast<float4 *>(ptab + (size_t)t * staged_slice_stride(BN)), SL4, pt,
+                             32 * PARTS);
             }
             BFMOE_TRACE(2, threadIdx.x == 64 && li == 0, 13);
             bool ok = mbar_wait(&tfull[b], (uint32_t)(li >> 1) & 1u);
@@ -447,7 +456,7 @@ __global__ void __launch_bounds__(contract_threads(BN), 1) k_contract(ContractPa
             const float scale = i >= 0 ? __uint_as_float(__ldg(p.packed + 2)) * p.gates[i] : 0.0f;
             const uint32_t tb = tmem + (uint32_t)(b * BN) + ((uint32_t)lane_base << 16);
             if (__all_sync(0xffffffffu, e == ea || e == eb)) {
-                const SmemTab st{smem_addr(ptab + (e == ea ? 0 : SIN * HB))};
+                const SmemTab st{smem_addr(ptab + (e == ea ? 0 : staged_slice_stride(BN)))};
                 epilogue_row<BN>(tb, st, out, scale, part, bar_id);
             } else {  // a third expert inside these 32 rows (a bucket of fewer than 32
                 // rows): every lane reads its own expert's table from global memory
