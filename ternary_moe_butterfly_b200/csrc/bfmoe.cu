@@ -227,7 +227,7 @@ struct StageRec {
     bool on = false;
 };
 
-const char *const kStageNames[] = {"route", "prep", "expert_in", "contract", "combine"};
+const char *const kStageNames[] = {"prep", "route", "expert_in", "contract", "combine"};
 constexpr int kNumStages = 5;
 
 void mark(StageRec *r, cudaStream_t st)
@@ -306,6 +306,35 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
 
     mark(rec, st);
 
+    PrepParams pp{};
+    pp.theta = theta;
+    pp.phi = phi;
+    pp.coef_t = ct;
+    pp.coef_p = cp;
+    pp.ncoef = N * L * (d / 2);
+    pp.d = d;
+    pp.L = L;
+    pp.packed = reinterpret_cast<const uint32_t *>(packed);
+    pp.wdec = wdec;
+    pp.status = status;
+    pp.x = x;
+    pp.x_bytes = (size_t)T_ * d * sizeof(T);
+    // one block per SM, beside the previous call's combine
+    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, sms));
+    void (*kp)(PrepParams) = nullptr;
+    switch (L) {
+    case 6: kp = k_prep<6>; break;
+    case 7: kp = k_prep<7>; break;
+    case 8: kp = k_prep<8>; break;
+    case 9: kp = k_prep<9>; break;
+    case 10: kp = k_prep<10>; break;
+    case 11: kp = k_prep<11>; break;
+    default: kp = k_prep<12>; break;
+    }
+    if (launch(kp, dim3(prep_grid), dim3(256), 0, st, rec == nullptr, false, pp) != cudaSuccess)
+        return BFMOE_ERR_CUDA;
+    mark(rec, st);
+
     RouteParams rp{};
     rp.logits = logits;
     rp.T = T_;
@@ -322,38 +351,9 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     rp.row_tok = row_tok;
     rp.row_exp = row_exp;
     rp.d = d;
+    rp.clear_status = 0;  // the prep kernel, first in the call, clears it
     bfmoe_status s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
-    mark(rec, st);
-
-    PrepParams pp{};
-    pp.theta = theta;
-    pp.phi = phi;
-    pp.coef_t = ct;
-    pp.coef_p = cp;
-    pp.ncoef = N * L * (d / 2);
-    pp.d = d;
-    pp.L = L;
-    pp.packed = reinterpret_cast<const uint32_t *>(packed);
-    pp.wdec = wdec;
-    pp.status = status;
-    pp.x = x;
-    pp.x_bytes = (size_t)T_ * d * sizeof(T);
-    // one block per SM: the prep shares the SMs with the routing, whose
-    // latency chain must keep most of the issue slots
-    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, sms));
-    void (*kp)(PrepParams) = nullptr;
-    switch (L) {
-    case 6: kp = k_prep<6>; break;
-    case 7: kp = k_prep<7>; break;
-    case 8: kp = k_prep<8>; break;
-    case 9: kp = k_prep<9>; break;
-    case 10: kp = k_prep<10>; break;
-    case 11: kp = k_prep<11>; break;
-    default: kp = k_prep<12>; break;
-    }
-    if (launch(kp, dim3(prep_grid), dim3(256), 0, st, rec == nullptr, false, pp) != cudaSuccess)
-        return BFMOE_ERR_CUDA;
     mark(rec, st);
 
     ExpertInParams ep{};
@@ -412,7 +412,7 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     cb.N = N;
     cb.s_lo = ilog2(BN);
     cb.topk_idx = idx;
-    cb.coef_p = cp;
+    cb.phi = phi;
     cb.y = y;
     cb.status = status;
     const int HS = L - cb.s_lo;
@@ -531,6 +531,7 @@ bfmoe_status bfmoe_route(const float *logits, int T, int N, int k, int32_t *topk
     rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
     rp.total = reinterpret_cast<int32_t *>(w + l.total);
     set_header(rp, w + l.status);
+    rp.clear_status = 1;
     s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
     return launched();
@@ -562,6 +563,7 @@ bfmoe_status bfmoe_route_static(const float *logits, int T, int N, int k, int32_
     rp.hist = reinterpret_cast<int32_t *>(w + l.hist);
     rp.total = reinterpret_cast<int32_t *>(w + l.total);
     set_header(rp, w + l.status);
+    rp.clear_status = 1;
     s = launch_route(rp, st);
     if (s != BFMOE_OK) return s;
     return launched();

@@ -333,7 +333,7 @@ struct CombineParams {
     int T, d, L, k, N;
     int s_lo;                 // first output stage left to apply (log2 of the GEMM's N tile)
     const int32_t *topk_idx;
-    const float2 *coef_p;     // [N][L*d/2] output table (see out_table_entry)
+    const float *phi;         // [N][L][d/2] output-butterfly angles
     void *y;
     uint32_t *status;
 };
@@ -382,18 +382,6 @@ __device__ __forceinline__ void load_halves(const __half *src, float *f)
     }
 }
 
-// n consecutive table entries (n even, 16-byte aligned) as n/2 16-byte loads
-template <int n>
-__device__ __forceinline__ void load_coef(const float2 *src, float2 *w)
-{
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-        const float4 f = __ldg(reinterpret_cast<const float4 *>(src) + i);
-        w[2 * i] = make_float2(f.x, f.y);
-        w[2 * i + 1] = make_float2(f.z, f.w);
-    }
-}
-
 // y_t = sum_j (stages s_lo..L-1 of B(phi_e)) slot_{t,j}: the rows arrive
 // already scaled by alpha * g.  HS = L - s_lo stages mix the NH = 2^HS slices
 // (pairs of slices nh, nh + 2^ls at the same in-slice column).  One thread per
@@ -412,7 +400,6 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
     constexpr int NH = 1 << HS;
     constexpr int M2 = BN / 32;
     constexpr int TPT = 4 * M2;  // threads per token
-    constexpr int PC = HS > 0 ? (HS << (HS - 1)) : 1;  // table entries per column
     constexpr int KB = KC > 0 ? KC : 1;                 // rows loaded together
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     const int t = tid / TPT;
@@ -445,39 +432,27 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
 #pragma unroll
             for (int b = 0; b < KB; ++b) {
                 if (HS > 0) {
-                    // combine part of the output table: [slot position][ls][pair over slices]
-                    const float2 *cf = p.coef_p + (size_t)ev[b] * p.L * half + (size_t)p.s_lo * half;
-                    if constexpr (PC == 1) {
-                        // one rotation per column: columns q, q+1 as a pair
-                        float2 w[QW];
-                        load_coef<QW>(cf + pos0 + q0, w);
+                    // stages s_lo + ls pair slices h, h + 2^ls at the same
+                    // in-slice column c: pair index c + BN * ri, with ri the
+                    // lower slice's index with bit ls deleted.  The angles come
+                    // straight from phi (no table: the next call's preparation
+                    // may already be rewriting the tables)
+                    const float *ph = p.phi + (size_t)ev[b] * p.L * half + (size_t)p.s_lo * half + col0 + q0;
 #pragma unroll
-                        for (int q = 0; q < QW; q += 2) {
-                            float2 a = make_float2(v[b][0][q], v[b][0][q + 1]);
-                            float2 c = make_float2(v[b][1][q], v[b][1][q + 1]);
-                            rot2(a, c, w[q], w[q + 1]);
-                            v[b][0][q] = a.x;
-                            v[b][0][q + 1] = a.y;
-                            v[b][1][q] = c.x;
-                            v[b][1][q + 1] = c.y;
+                    for (int ls = 0; ls < HS; ++ls)
+#pragma unroll
+                        for (int ri = 0; ri < NH / 2; ++ri) {
+                            const int h = insert_zero_bit(ri, ls);
+                            float a[QW];
+#pragma unroll
+                            for (int q = 0; q < QW; ++q) a[q] = __ldg(ph + (size_t)ls * half + BN * ri + q);
+#pragma unroll
+                            for (int q = 0; q < QW; ++q) {
+                                float sn, cs;
+                                __sincosf(a[q], &sn, &cs);
+                                rot1(v[b][h][q], v[b][h + (1 << ls)][q], cs, sn);
+                            }
                         }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < QW; ++q) {
-                            float2 w[PC];
-                            load_coef<PC>(cf + (size_t)(pos0 + q0 + q) * PC, w);
-                            const float *wf = reinterpret_cast<const float *>(w);
-#pragma unroll
-                            for (int ls = 0; ls < HS; ++ls)
-#pragma unroll
-                                for (int ri = 0; ri < NH / 2; ++ri) {
-                                    const int h = insert_zero_bit(ri, ls);
-                                    const int r = (ls << (HS > 0 ? HS - 1 : 0)) + ri;
-                                    rot1(v[b][h][q], v[b][h + (1 << ls)][q], wf[4 * (r >> 1) + (r & 1)],
-                                         wf[4 * (r >> 1) + 2 + (r & 1)]);
-                                }
-                        }
-                    }
                 }
 #pragma unroll
                 for (int h = 0; h < NH; ++h)

@@ -1,12 +1,13 @@
-// prep.cuh -- per-call preparation of the layer's weights, run beside the
-// routing: the butterfly angles become {cos, sin} tables in the order the
-// kernels consume them, and the 2-bit packed base becomes the tensor-core
-// operand layout.
+// prep.cuh -- per-call preparation of the layer's weights, the first
+// kernel of a forward: the butterfly angles become {cos, sin} tables in the
+// order the kernels consume them, and the 2-bit packed base becomes the
+// tensor-core operand layout.
 //
-// The prep kernel is launched with a programmatic dependency on the
-// cooperative routing kernel, which lets it start at once: it uses the SM
-// resources the routing leaves free, and ends by waiting for the routing to
-// complete, so that the kernels after it see both results.
+// It is launched with a programmatic dependency on the previous call's last
+// kernel (the combine, which reads no table), so it runs while that kernel
+// finishes: nothing it writes is read by the previous call's combine, and it
+// waits for that call to complete only at its end, before it clears the
+// status word.  The routing kernel depends on it in turn.
 #pragma once
 
 #include "butterfly.cuh"
@@ -40,8 +41,8 @@ struct PrepParams {
 template <int LL>
 __global__ void __launch_bounds__(256) k_prep(PrepParams p)
 {
-    // the input-butterfly kernel may become resident now; it still waits for
-    // this grid (and so for the routing) to complete before reading anything
+    // the routing kernel may become resident now; it waits for this grid
+    // to complete before it touches the workspace
     BFMOE_TRACE(4, threadIdx.x == 0, 0);
     pdl_trigger();
     if (threadIdx.x == 0 && p.x) {
@@ -103,11 +104,15 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
         }
     }
     BFMOE_TRACE(4, threadIdx.x == 0, 1);
-    if (gtid == 0 && (p.packed[0] != kPackMagic || p.packed[1] != (uint32_t)d)) set_status(p.status, BFMOE_ERR_INVALID_ARG);
+    const bool bad_header = gtid == 0 && (p.packed[0] != kPackMagic || p.packed[1] != (uint32_t)d);
     constexpr int nq = d * d / 8;
     for (int q = gtid; q < nq; q += gthreads) decode_chunk(p.packed, d, p.wdec, q);
     BFMOE_TRACE(4, threadIdx.x == 0, 2);
-    pdl_wait();  // complete only after the routing has
+    // complete only after the previous call on this stream has (its last
+    // kernels may still read the routing results this call overwrites);
+    // then this call's status starts clear
+    pdl_wait();
+    if (gtid == 0) *reinterpret_cast<volatile uint32_t *>(p.status) = bad_header ? (uint32_t)BFMOE_ERR_INVALID_ARG : 0u;
     BFMOE_TRACE(4, threadIdx.x == 0, 3);
 }
 

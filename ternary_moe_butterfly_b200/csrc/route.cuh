@@ -63,6 +63,7 @@ struct RouteParams {
     // forward only: the bucket rows' tokens and experts for the input butterfly
     int32_t *row_tok;    // [T*k] token of each bucket row, or null
     int32_t *row_exp;    // [T*k] expert of each bucket row, or null
+    int clear_status;    // the routing starts the call: it clears the status word
 };
 
 // Histogram budget of the route kernel's shared memory, and the number of
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         // a new call's status; every other status write of this launch comes
         // after the grid barrier, which block 0 reaches after this store
-        *reinterpret_cast<volatile uint32_t *>(p.status) = 0u;
+        if (p.clear_status) *reinterpret_cast<volatile uint32_t *>(p.status) = 0u;
         grid_epoch_open(p.sync, p.departed, p.epoch, p.token);
     }
     // ---- phase A: top-k over this block's token range
@@ -448,8 +449,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
         grid_depart(p.sync, p.departed, nblk);
         return;
     }
-    // the prep kernel may start now and run beside the rest of the routing
-    // (earlier, it slows the top-k and the barrier more than it gains)
+    // the input-butterfly kernel may become resident now (earlier, its
+    // blocks would crowd the routing's)
     pdl_trigger();
     if (nan_here && threadIdx.x == 0) set_status(p.status, BFMOE_ERR_NONFINITE);
     BFMOE_TRACE(0, threadIdx.x == 0, 3);
