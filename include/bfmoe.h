@@ -53,6 +53,16 @@
  * separate copy.  Calls that share a workspace must be ordered (one stream,
  * or events).
  *
+ * Launch overlap: the kernels of a call are chained with programmatic
+ * dependent launch, and bfmoe_forward's first kernel (the weight
+ * preparation) may start as soon as the previous kernel on the stream allows
+ * its dependents to launch.  It reads theta, phi and the packed base before
+ * it waits for that kernel; everything else (x, logits, workspace) is read
+ * only after the wait.  So the kernel just before a forward must not write
+ * theta, phi or the packed base if it triggers its dependents early
+ * (griddepcontrol.launch_dependents); kernels that never do, and any
+ * event, copy or other kernel in between, keep plain stream order.
+ *
  * Limits: d is a power of two in [64, 4096]; 1 <= N <= 4096;
  * 1 <= k <= min(N, 8); 1 <= T <= 2^24 / k; x and y are fp32 or bf16,
  * 16-byte aligned; workspaces are 256-byte aligned.
