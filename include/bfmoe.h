@@ -56,9 +56,11 @@
  * Launch overlap: the kernels of a call are chained with programmatic
  * dependent launch, and bfmoe_forward's first kernel (the weight
  * preparation) may start as soon as the previous kernel on the stream allows
- * its dependents to launch.  It reads theta, phi and the packed base before
- * it waits for that kernel; everything else (x, logits, workspace) is read
- * only after the wait.  So the kernel just before a forward must not write
+ * its dependents to launch.  It reads theta, phi and the packed base (and
+ * writes the workspace's cos/sin tables and decoded base, which only this
+ * call's later kernels read) before it waits for that kernel; x, the logits
+ * and the routing results are touched only after the wait (x is merely
+ * prefetched into L2 before it).  So the kernel just before a forward must not write
  * theta, phi or the packed base if it triggers its dependents early
  * (griddepcontrol.launch_dependents); kernels that never do, and any
  * event, copy or other kernel in between, keep plain stream order.
