@@ -65,20 +65,26 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
     constexpr int tab = L * half;
     const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
     const int gthreads = gridDim.x * blockDim.x;
-    // rotation pairs: [0, ncoef/2) of the input table, then the output table
-    const int npair = p.ncoef;
+    // rotation pairs: the input table, then the output table's slice part
+    // (its combine part is not written: the combine reads phi itself)
+    constexpr int used = slice_stages(gemm_bn(d)) * half;  // output rotations per expert
+    const int nexp = p.ncoef / tab;
+    const int npair_in = p.ncoef / 2, npair = npair_in + nexp * (used / 2);
     for (int j0 = gtid; j0 < npair; j0 += 2 * gthreads) {
         float a[2][2];
         int dst[2];
+        bool outt[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int j = j0 + u * gthreads;
             dst[u] = -1;
+            outt[u] = false;
             a[u][0] = a[u][1] = 0.0f;
             if (j < npair) {
-                const bool out = j >= p.ncoef / 2;
-                const int jj = out ? j - p.ncoef / 2 : j;
-                const int e = (2 * jj) / tab, r = (2 * jj) % tab;
+                const bool out = j >= npair_in;
+                const int jj = out ? j - npair_in : j;
+                const int per = out ? used : tab;
+                const int e = (2 * jj) / per, r = (2 * jj) % per;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     int st, pp;
@@ -88,7 +94,8 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
                         engine_entry(d, L, true, r + h, st, pp);
                     a[u][h] = __ldg((out ? p.phi : p.theta) + (size_t)e * tab + st * half + pp);
                 }
-                dst[u] = j;
+                dst[u] = (e * tab + r) / 2;  // float4 index of the pair
+                outt[u] = out;
             }
         }
 #pragma unroll
@@ -97,8 +104,8 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
             float s0, c0, s1, c1;
             __sincosf(a[u][0], &s0, &c0);
             __sincosf(a[u][1], &s1, &c1);
-            if (dst[u] >= p.ncoef / 2)
-                reinterpret_cast<float4 *>(p.coef_p)[dst[u] - p.ncoef / 2] = make_float4(c0, c1, s0, s1);
+            if (outt[u])
+                reinterpret_cast<float4 *>(p.coef_p)[dst[u]] = make_float4(c0, c1, s0, s1);
             else
                 reinterpret_cast<float4 *>(p.coef_t)[dst[u]] = make_float4(c0, c1, -s0, -s1);
         }
