@@ -150,21 +150,22 @@ def dist_env():
 
 # ----------------------------------------------------------------- reference
 
-def cpu_oracle_rate(w: wl.Workload, target_s: float, inp=None, max_tokens=None):
-    """tokens/s of the fp64 oracle on the host cores over a bounded sample."""
+def cpu_oracle_rate(w: wl.Workload, target_s: float, inp=None, max_tokens=None, nthreads: int = 0):
+    """tokens/s of the fp64 oracle on the host cores over a bounded sample
+    (nthreads OpenMP threads; 0: all the runtime offers)."""
     import oracle
     inp = inp or wl.make_inputs(w.name, T=min(w.T, 64))
-    threads = oracle.max_threads()
+    threads = nthreads if nthreads > 0 else oracle.max_threads()
     n = min(16, inp.x.shape[0])
     t0 = time.perf_counter()
-    oracle.forward(inp.x[:n], inp.logits[:n], w.k, inp.w_base, inp.alpha, inp.theta, inp.phi)
+    oracle.forward(inp.x[:n], inp.logits[:n], w.k, inp.w_base, inp.alpha, inp.theta, inp.phi, nthreads=threads)
     per_tok = max((time.perf_counter() - t0) / n, 1e-6)
     n2 = int(max(n, min(1 << 20 if max_tokens is None else max_tokens, target_s / per_tok)))
     reps = max(1, int(math.ceil(n2 / inp.x.shape[0])))
     xs = np.concatenate([inp.x] * reps)[:n2]
     ls = np.concatenate([inp.logits] * reps)[:n2]
     t0 = time.perf_counter()
-    oracle.forward(xs, ls, w.k, inp.w_base, inp.alpha, inp.theta, inp.phi)
+    oracle.forward(xs, ls, w.k, inp.w_base, inp.alpha, inp.theta, inp.phi, nthreads=threads)
     dt = time.perf_counter() - t0
     return n2 / dt, threads, n2, dt
 
@@ -363,6 +364,10 @@ def run_ours(args, w):
         "route": ("hbm", T * N * 4 + T * k * 12, "GB/s"),
     }
     dom = max(prof, key=prof.get) if prof else None
+    # rows per expert of the last forward on this workspace (skewed loads show here)
+    _, _, _, offs = bf.forward_routing(ws, T, d, N, k)
+    sizes = np.diff(offs.cpu().numpy().astype(np.int64))
+    buckets = {"max": int(sizes.max()), "min": int(sizes.min()), "empty": int((sizes == 0).sum())}
     roof = None
     if dom in models:
         bound, amount, unit = models[dom]
@@ -385,6 +390,10 @@ def run_ours(args, w):
         r, threads, n, dt = cpu_oracle_rate(w, args.cpu_seconds)
         cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens of the {w.name} workload, fp64 C oracle with OpenMP, {dt:.1f} s"}
+        if w.name in ("tiny", "headline"):
+            r1, _, n1, dt1 = cpu_oracle_rate(w, min(2.0, args.cpu_seconds / 4), nthreads=1)
+            cpu["single_thread_value"] = r1
+            cpu["single_thread_sample"] = f"{n1} tokens, 1 thread, {dt1:.1f} s"
 
     if rank == 0:
         line = {
@@ -399,7 +408,13 @@ def run_ours(args, w):
             "layer_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms * 1e3, "frac": t_roof / (ms * 1e-3),
                                "bound": "tensor" if t_tensor >= t_hbm else "hbm",
                                "t_tensor_us": t_tensor * 1e6, "t_hbm_us": t_hbm * 1e6,
-                               "peaks": f"{peaks['bf16_tflops']} TF bf16, {peaks['hbm_gbs']} GB/s ({peaks['source']})"},
+                               "frac_sustained": max(flops / (peaks.get("bf16_tflops_sustained",
+                                                                        peaks["bf16_tflops"]) * 1e12),
+                                                     t_hbm) / (ms * 1e-3),
+                               "peaks": f"{peaks['bf16_tflops']} TF bf16 burst, "
+                                        f"{peaks.get('bf16_tflops_sustained', peaks['bf16_tflops'])} TF sustained, "
+                                        f"{peaks['hbm_gbs']} GB/s ({peaks['source']})"},
+            "buckets": buckets,
             "roofline": roof,
             "kernels_ms": prof,
             "gpu_launches": len(prof) * ksteps if prof else None,
