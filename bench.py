@@ -148,6 +148,30 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest of the ranks' values (every rank takes part); x itself
+    without an initialised process group of more than one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(w: wl.Workload, rank: int) -> int:
+    """Each rank routes its own tokens (weak scaling: replicas of the layer,
+    disjoint synthetic token shards)."""
+    return w.seed + 1000 * rank
+
+
+def job_tokens_per_s(world: int, T: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's T tokens per step over the slowest
+    rank's step time."""
+    return world * T / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------- reference
 
 def cpu_oracle_rate(w: wl.Workload, target_s: float, inp=None, max_tokens=None, nthreads: int = 0):
@@ -222,7 +246,7 @@ def run_ours(args, w):
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
 
-    inp = wl.make_inputs(w.name, seed=w.seed + 1000 * rank)
+    inp = wl.make_inputs(w.name, seed=rank_seed(w, rank))
     d, N, k, T = w.d, w.N, w.k, w.T
     xdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     xb = 2 if w.dtype == "bf16" else 4
@@ -290,10 +314,7 @@ def run_ours(args, w):
     st = bf.sync_status(ws, stream)
     if st != bf.OK:
         raise RuntimeError(f"timed status {bf.status_string(st)}")
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device)
 
     # per-kernel durations (events between the launches of one step)
     prof = {}
@@ -338,11 +359,7 @@ def run_ours(args, w):
         g2.replay()
         f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / K
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / K, device)
     if bf.sync_status(ws, stream) != bf.OK:
         raise RuntimeError("e2e status")
 
@@ -350,7 +367,7 @@ def run_ours(args, w):
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = bmin / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_tensor, t_hbm)
-    value = world * T / (ms * 1e-3)
+    value = job_tokens_per_s(world, T, ms)
 
     # dominant kernel and its roofline
     R, Rp, L = T * k, (T * k + 127) // 128 * 128, w.L
@@ -419,7 +436,7 @@ def run_ours(args, w):
             "kernels_ms": prof,
             "gpu_launches": len(prof) * ksteps if prof else None,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": job_tokens_per_s(world, T, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size() + ls[0].numel() * 4),
                     "d2h_bytes_per_step": int(ys[0].numel() * ys[0].element_size()), "ms_per_step": e2e_ms},
             "clocks": clocks,
