@@ -20,7 +20,7 @@
 //            output-butterfly stages that stay inside the slice
 //            (stages 0 .. log2 BN - 1) to its own row, with the row's expert
 //            table, scales by alpha * gate and stores fp16 to the row's
-//            token-order slot (the slot layout below).
+//            token-order slot (the slot layout described with CombineParams).
 //            Stages 0-4 act inside 32-column blocks (one 32-column TMEM load,
 //            rotate, store back); stages 5.. act on columns 32 apart (4-column
 //            TMEM loads).  The remaining stages, which mix slices, are

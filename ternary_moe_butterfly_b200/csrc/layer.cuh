@@ -1,10 +1,13 @@
 // layer.cuh -- the expert-layer kernels around the contraction:
 //   k_pack_base    int8 ternary W_base -> 2-bit packed words
-//   k_expert_in    gather each single-expert tile of bucketed rows, input
-//                  rotation B(theta_e)^T, fp16 operand blocks for the GEMM
+//   k_expert_in    gather each 32-row tile of bucketed rows (one or two
+//                  experts' tables staged, else read from global memory),
+//                  input rotation B(theta_e)^T, fp16 operand blocks for the
+//                  GEMM
 //   k_combine      output stages the GEMM epilogue could not reach (those
-//                  that mix columns 256 or more apart), alpha * gate, and
-//                  the per-token sum over the k routed rows
+//                  that mix columns 256 or more apart, angles read from phi)
+//                  and the per-token sum over the k routed rows, which the
+//                  epilogue already scaled by alpha * gate
 //   k_bfly_apply   standalone row butterfly (B or B^T)
 //
 // The method: expert i is W_i = alpha B(phi_i) W_base B(theta_i)^T with a
