@@ -334,6 +334,19 @@ __global__ void __launch_bounds__(contract_threads(BN), 1) k_contract(ContractPa
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     BFMOE_TRACE(2, threadIdx.x == 0, 1);
+    // The W operand blocks were decoded by the prep kernel, which completed
+    // before the input-butterfly kernel (this grid's predecessor) could
+    // start: the producer streams the first stages' W blocks before it
+    // waits.  Everything else waits for the input kernel (the A blocks).
+    const bool early_w = warp == 0 && lane == 0 && (int)blockIdx.x < nunits;
+    const int npre = early_w ? (KC < kStages ? KC : kStages) : 0;
+    if (early_w) {
+        const __half *b_src = p.w_blocks + (size_t)(blockIdx.x % NH) * KC * ((size_t)BN * kBK);
+        for (int kc = 0; kc < npre; ++kc) {
+            mbar_arrive_expect_tx(&full[kc], a_bytes + b_bytes);
+            bulk_g2s(sB + (size_t)kc * b_bytes, b_src + (size_t)kc * ((size_t)BN * kBK), b_bytes, &full[kc]);
+        }
+    }
     pdl_wait();  // the A blocks come from the input-butterfly kernel
     pdl_trigger();
     BFMOE_TRACE(2, threadIdx.x == 0, 2);
@@ -348,6 +361,11 @@ __global__ void __launch_bounds__(contract_threads(BN), 1) k_contract(ContractPa
                 for (int kc = 0; kc < KC; ++kc, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    if (it < npre) {  // its W block is already on the way
+                        BFMOE_TRACE(2, it == 0, 3);
+                        bulk_g2s(sA + (size_t)s * a_bytes, a_src + (size_t)kc * (kBM * kBK), a_bytes, &full[s]);
+                        continue;
+                    }
                     if (!mbar_wait(&empty[s], ph ^ 1u)) {
                         set_status(p.status, BFMOE_ERR_TIMEOUT);
                         *abort_flag = 1;

@@ -28,7 +28,26 @@ struct PrepParams {
     uint32_t *status;
     const void *x;             // layer input, prefetched into L2 ([x_bytes], 16-byte multiple)
     size_t x_bytes;
+    const void *logits;        // router logits, prefetched into L2 ([logit_bytes])
+    size_t logit_bytes;
 };
+
+// Bring block `blk` of `nblk`'s share of [base, base + bytes) into L2 (one
+// thread; shares rounded to 16 bytes, the prefetch unit; `bytes` a multiple
+// of 16; nothing for a base that is not 16-byte aligned).
+__device__ __forceinline__ void l2_prefetch_share(const void *base, size_t bytes, int blk, int nblk)
+{
+    const size_t share = ((bytes + nblk - 1) / nblk + 15) & ~size_t(15);
+    const size_t lo = (size_t)blk * share;
+    if (!base || (reinterpret_cast<uintptr_t>(base) & 15) || lo >= bytes) return;  // 16-byte rule
+    const size_t n = bytes - lo < share ? bytes - lo : share;
+    for (size_t o = 0; o < n; o += (1u << 20)) {
+        const uint32_t c = (uint32_t)(n - o < (1u << 20) ? n - o : (1u << 20));
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<const char *>(base) + lo + o),
+                     "r"(c)
+                     : "memory");
+    }
+}
 
 // {cos, sin} tables of every expert in consumption order: theta -> the
 // input engine's B^T table (engine_entry order, sign of B^T folded in), phi
@@ -45,21 +64,13 @@ __global__ void __launch_bounds__(256) k_prep(PrepParams p)
     // to complete before it touches the workspace
     BFMOE_TRACE(4, threadIdx.x == 0, 0);
     pdl_trigger();
-    if (threadIdx.x == 0 && p.x) {
-        // the input-butterfly kernel gathers x right after the routing: bring
-        // this block's share of it into L2 now (off the routing's path)
-        const size_t share = ((p.x_bytes + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
-        const size_t lo = (size_t)blockIdx.x * share;
-        if (lo < p.x_bytes) {
-            const size_t n = p.x_bytes - lo < share ? p.x_bytes - lo : share;
-            for (size_t o = 0; o < n; o += (1u << 20)) {
-                const uint32_t c = (uint32_t)(n - o < (1u << 20) ? n - o : (1u << 20));
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                                 reinterpret_cast<const char *>(p.x) + lo + o),
-                             "r"(c)
-                             : "memory");
-            }
-        }
+    if (threadIdx.x == 0) {
+        // the routing reads the logits and the input kernel gathers x right
+        // after this kernel: bring this block's shares into L2 now (a
+        // prefetch reads nothing into the program, so it may run before the
+        // wait for the previous kernel)
+        l2_prefetch_share(p.logits, p.logit_bytes, blockIdx.x, gridDim.x);
+        l2_prefetch_share(p.x, p.x_bytes, blockIdx.x, gridDim.x);
     }
     constexpr int L = LL, d = 1 << LL, half = d >> 1;
     constexpr int tab = L * half;
