@@ -321,8 +321,8 @@ bfmoe_status launch_layer(const void *x, int T_, int d, int N, int k, const void
     pp.x_bytes = (size_t)T_ * d * sizeof(T);
     pp.logits = logits;
     pp.logit_bytes = ((size_t)T_ * N * 4) & ~size_t(15);
-    // one block per SM, beside the previous call's combine
-    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, sms));
+    // two blocks per SM, beside the previous call's combine
+    const int prep_grid = std::max(1, std::min((2 * pp.ncoef + 255) / 256, 2 * sms));
     void (*kp)(PrepParams) = nullptr;
     switch (L) {
     case 6: kp = k_prep<6>; break;
