@@ -240,10 +240,17 @@ __global__ void __launch_bounds__(kInThreads, 2) k_expert_in(ExpertInParams p)
             }
             if (lane == 0) *mode = two ? 1 : 0;
         }
-        const bool ok = __syncthreads_and(mbar_wait(bar, phase));
+        const uint32_t cur = phase;
+        const bool ok = __syncthreads_and(mbar_wait(bar, cur));
         phase ^= 1;
         if (!ok) {
-            if (threadIdx.x == 0) set_status(p.status, BFMOE_ERR_TIMEOUT);
+            if (threadIdx.x == 0) {
+                set_status(p.status, BFMOE_ERR_TIMEOUT);
+                // the copies of this tile must land before the block's
+                // shared memory is released: one more bounded wait
+                mbar_wait(bar, cur);
+            }
+            __syncthreads();
             break;
         }
         const bool two = *mode != 0;
