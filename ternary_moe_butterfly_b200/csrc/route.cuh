@@ -150,10 +150,9 @@ __device__ __forceinline__ void grid_depart(uint32_t *ctr, uint32_t *departed, i
 __device__ __forceinline__ void grid_arrive(uint32_t *ctr)
 {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
-    }
+    // a release add: the block's earlier writes (ordered before this thread
+    // by the barrier) become visible before the count does
+    if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 
 __device__ bool grid_wait(uint32_t *ctr, uint32_t target, uint32_t *status)
@@ -163,15 +162,15 @@ __device__ bool grid_wait(uint32_t *ctr, uint32_t target, uint32_t *status)
         ok = 1;
         const unsigned long long t0 = globaltimer_ns();
         while (true) {
-            const uint32_t v = *reinterpret_cast<volatile uint32_t *>(ctr);
-            if (v >= target) break;
+            uint32_t v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= target) break;  // the acquire orders the other blocks' writes before ours
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 set_status(status, BFMOE_ERR_TIMEOUT);
                 ok = 0;
                 break;
             }
         }
-        __threadfence();
     }
     __syncthreads();
     return ok != 0;
