@@ -404,15 +404,22 @@ template <typename T, int HS, int BN, int QW, int KC>
 __global__ void __launch_bounds__(256) k_combine(CombineParams p)
 {
     BFMOE_TRACE(3, threadIdx.x == 0, 0);
-    pdl_wait();
-    BFMOE_TRACE(3, threadIdx.x == 0, 1);
-    pdl_trigger();
     constexpr int NH = 1 << HS;
     constexpr int M2 = BN / 32;
     constexpr int TPT = 4 * M2;  // threads per token
     constexpr int KB = KC > 0 ? KC : 1;                 // rows loaded together
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
     const int t = tid / TPT;
+    // with k fixed, the rows' expert indices are read before the wait (the
+    // routing finished before the kernel this grid depends on started), so
+    // that after it the products and the angles load together
+    int ev_pre[KB];
+#pragma unroll
+    for (int b = 0; b < KB; ++b)
+        ev_pre[b] = (KC > 0 && HS > 0 && t < p.T) ? min(max(__ldg(p.topk_idx + t * KB + b), 0), p.N - 1) : 0;
+    pdl_wait();
+    BFMOE_TRACE(3, threadIdx.x == 0, 1);
+    pdl_trigger();
     if (t >= p.T) return;
     const int k = KC > 0 ? KC : p.k;
     const int g = (tid % TPT) / M2, m = tid % M2;
@@ -434,7 +441,7 @@ __global__ void __launch_bounds__(256) k_combine(CombineParams p)
 #pragma unroll
             for (int b = 0; b < KB; ++b) {
                 const int i = t * k + j0 + b;
-                ev[b] = HS > 0 ? min(max(__ldg(p.topk_idx + i), 0), p.N - 1) : 0;
+                ev[b] = HS == 0 ? 0 : (KC > 0 ? ev_pre[b] : min(max(__ldg(p.topk_idx + i), 0), p.N - 1));
                 const __half *row = p.slot + (size_t)i * d + pos0 + q0;
 #pragma unroll
                 for (int h = 0; h < NH; ++h) load_halves<QW>(row + h * BN, v[b][h]);
