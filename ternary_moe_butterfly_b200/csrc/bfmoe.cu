@@ -58,8 +58,9 @@ bfmoe_status check_route_shape(int T, int N, int k)
 // Rows of the per-block histogram (the routing grid never exceeds it).
 int route_chunks(int) { return kMaxRouteBlocks; }
 
-// Status word and grid-barrier counter share the first 16 bytes of every
-// workspace; one memset clears both.
+// Every workspace opens with the 32-byte header (status word, grid-barrier
+// and departure counters, launch epoch) in its first aligned slot; the
+// barrier words clear themselves, so no call issues a memset.
 struct RouteLayout {
     size_t status, hist, total, total_bytes;
 };

@@ -69,7 +69,11 @@ struct RouteParams {
 // Histogram budget of the route kernel's shared memory, and the number of
 // selected experts of its own rows a block keeps for the scatter.
 constexpr int kSelCap = 2048;
-constexpr int kLogitStageInts = 10240;  // staged logits per batch (40 KB)
+
+// Staged logits per batch: 40 KB, or 120 KB above 128 experts (a block's
+// token range then still fits in one batch at the usual sizes, so its
+// loads take two rounds rather than two per batch).
+__host__ __device__ constexpr int route_stage_ints(int N) { return N > 128 ? 30720 : 10240; }
 
 // Padded shared-memory row of one token's logits when `grp` lanes share
 // the token: rows G floats apart on top of a 32-float multiple put the group's
@@ -80,7 +84,7 @@ __host__ __device__ inline int logit_row_stride(int N, int grp) { return grp < 3
 // the widest row stride (16 lanes per token).
 __host__ __device__ inline int route_batch_tokens(int N)
 {
-    const int b = kLogitStageInts / logit_row_stride(N, 16);
+    const int b = route_stage_ints(N) / logit_row_stride(N, 16);
     return b < 1 ? 1 : (b > 256 ? 256 : b);
 }
 
@@ -288,15 +292,16 @@ __device__ void topk_range(const RouteParams &p, int t0, int t1, int *sh_hist, f
         if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0) {
             const float4 *s4 = reinterpret_cast<const float4 *>(src);
             const int n4 = (int)(nval / 4);
-            for (int q0 = threadIdx.x; q0 < n4; q0 += 8 * blockDim.x) {
-                float4 v[8];
+            constexpr int kRound = 16;  // 16-byte loads in flight per thread
+            for (int q0 = threadIdx.x; q0 < n4; q0 += kRound * blockDim.x) {
+                float4 v[kRound];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < kRound; ++u) {
                     const int qq = q0 + u * blockDim.x;
                     if (qq < n4) v[u] = __ldg(s4 + qq);
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < kRound; ++u) {
                     const int qq = q0 + u * blockDim.x;
                     if (qq >= n4) break;
                     const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -372,9 +377,13 @@ __device__ __forceinline__ void decode_chunk(const uint32_t *__restrict__ packed
     reinterpret_cast<uint4 *>(wb)[q] = make_uint4(h[0], h[1], h[2], h[3]);
 }
 
+// Partial sums of the histogram read, per half: parts * N <= 4 * threads
+// (see the one-barrier read in k_route).
+constexpr int kRouteRedInts = 4 * kRouteThreads;
+
 // Shared-memory plan of the route kernel, in ints: the kept experts of the
-// block's rows, then either phase A (histogram + staged logits) or phases
-// B/C (offsets, bucket bases, partial sums), 16-byte aligned.
+// block's rows, then either phase A (histogram + staged logits, the latter
+// 16-byte aligned) or phases B/C (offsets, bucket bases, partial sums).
 struct RouteSmem {
     int keep, a_hist, a_logits, off, cnt, red, total;
     __host__ __device__ explicit RouteSmem(int N)
@@ -383,11 +392,11 @@ struct RouteSmem {
         keep = 0;
         a_hist = kSelCap;
         a_logits = a_hist + np4;
-        const int a_end = a_logits + kLogitStageInts;
+        const int a_end = a_logits + route_stage_ints(N);
         off = kSelCap;
         cnt = off + N + 1;
         red = cnt + N;
-        const int c_end = red + 2 * kRouteThreads;
+        const int c_end = red + 2 * kRouteRedInts;
         total = a_end > c_end ? a_end : c_end;
     }
 };
@@ -459,28 +468,57 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(RouteParams p)
     if (one_barrier) {
         // ---- every block: expert totals and its own prefix over the blocks
         // before it, straight from the block-major histogram: `parts`
-        // threads per expert take every parts-th row (a warp reads 32
-        // consecutive experts of a row), 32 loads in flight per thread
+        // threads per expert (or per 4 experts, with 16-byte loads when N is
+        // a multiple of 4: the rows are then 16-byte aligned and unpadded)
+        // take every parts-th row, many loads in flight per thread.
+        // parts * N <= 4 * blockDim.x either way.
         int *red = sh + lay.red;  // [2][parts * N]
-        const int parts = max(1, (int)blockDim.x / N);
-        for (int idx = threadIdx.x; idx < parts * N; idx += blockDim.x) {
-            const int e = idx % N, part = idx / N;
-            int tot = 0, pre = 0;
-            for (int b0 = part; b0 < nblk; b0 += 32 * parts) {
-                int v[32];
+        const bool by4 = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(p.hist) & 15) == 0;
+        const int cols = by4 ? N >> 2 : N;
+        const int parts = max(1, (int)blockDim.x / cols);
+        if (by4) {
+            const int4 *h4 = reinterpret_cast<const int4 *>(p.hist);
+            for (int idx = threadIdx.x; idx < parts * cols; idx += blockDim.x) {
+                const int c = idx % cols, part = idx / cols;
+                int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+                for (int b0 = part; b0 < nblk; b0 += 16 * parts) {
+                    int4 v[16];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int b = b0 + u * parts;
-                    v[u] = b < nblk ? __ldcg(p.hist + (size_t)b * np4 + e) : 0;
-                }
+                    for (int u = 0; u < 16; ++u) {
+                        const int b = b0 + u * parts;
+                        v[u] = b < nblk ? __ldcg(h4 + (size_t)b * cols + c) : make_int4(0, 0, 0, 0);
+                    }
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    tot += v[u];
-                    pre += (b0 + u * parts < (int)blockIdx.x) ? v[u] : 0;
+                    for (int u = 0; u < 16; ++u) {
+                        tot.x += v[u].x, tot.y += v[u].y, tot.z += v[u].z, tot.w += v[u].w;
+                        if (b0 + u * parts < (int)blockIdx.x)
+                            pre.x += v[u].x, pre.y += v[u].y, pre.z += v[u].z, pre.w += v[u].w;
+                    }
                 }
+                int *rt = red + part * N + 4 * c, *rp = rt + parts * N;
+                rt[0] = tot.x, rt[1] = tot.y, rt[2] = tot.z, rt[3] = tot.w;
+                rp[0] = pre.x, rp[1] = pre.y, rp[2] = pre.z, rp[3] = pre.w;
             }
-            red[idx] = tot;
-            red[parts * N + idx] = pre;
+        } else {
+            for (int idx = threadIdx.x; idx < parts * N; idx += blockDim.x) {
+                const int e = idx % N, part = idx / N;
+                int tot = 0, pre = 0;
+                for (int b0 = part; b0 < nblk; b0 += 32 * parts) {
+                    int v[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int b = b0 + u * parts;
+                        v[u] = b < nblk ? __ldcg(p.hist + (size_t)b * np4 + e) : 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        tot += v[u];
+                        pre += (b0 + u * parts < (int)blockIdx.x) ? v[u] : 0;
+                    }
+                }
+                red[idx] = tot;
+                red[parts * N + idx] = pre;
+            }
         }
         __syncthreads();
         BFMOE_TRACE(0, threadIdx.x == 0, 6);
