@@ -177,6 +177,46 @@ def _ptr(t):
     return None if t is None else int(t.data_ptr())
 
 
+def _need(t, name, dtype=None, dims=None, numel=None, min_numel=None):
+    """t must be passable to the C ABI as a plain pointer: a contiguous
+    tensor of the given dtype, rank and size (the device is checked by
+    _on_device once every argument has passed)."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs at least {min_numel}")
+    return t
+
+
+def _on_device(first, **others):
+    """Every tensor argument on one CUDA device (the kernels dereference
+    the pointers there); returns that device."""
+    dev = first.device
+    if dev.type != "cuda":
+        raise ValueError(f"the arguments must be CUDA tensors, got one on {dev}")
+    for name, t in others.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other arguments on {dev}")
+    return dev
+
+
+def _angle_count(N, d):
+    """Elements of an angle table [N][log2 d][d/2] (None when d is not a
+    power of two: the C call rejects that width)."""
+    if d < 2 or d & (d - 1):
+        return None
+    return N * (d.bit_length() - 1) * (d // 2)
+
+
 def _check(code, what):
     if code != OK:
         raise BfmoeError(code, what)
@@ -190,17 +230,24 @@ def _ws(nbytes, device):
 def pack_base(w, alpha: float, stream=None):
     """int8 [d][d] ternary (device) -> packed uint8 tensor (synchronises)."""
     torch = _torch()
+    if not isinstance(w, torch.Tensor) or w.dim() != 2 or w.shape[0] != w.shape[1]:
+        raise ValueError("w must be a square [d][d] tensor")
+    w = _need(w.contiguous(), "w", torch.int8)
+    dev = _on_device(w)
     d = int(w.shape[0])
-    out = torch.empty(max(int(bfmoe_packed_base_bytes(d)), 16), dtype=torch.uint8, device=w.device)
-    _check(bfmoe_pack_base(_ptr(w.contiguous()), d, float(alpha), _ptr(out), _stream(stream)), "bfmoe_pack_base")
+    out = torch.empty(max(int(bfmoe_packed_base_bytes(d)), 16), dtype=torch.uint8, device=dev)
+    _check(bfmoe_pack_base(_ptr(w), d, float(alpha), _ptr(out), _stream(stream)), "bfmoe_pack_base")
     return out
 
 
 def route(logits, k: int, ws=None, stream=None):
     """Top-k routing and bucketing; returns (topk_idx, gates, perm, offsets, ws)."""
     torch = _torch()
+    _need(logits, "logits", torch.float32, dims=2)
     T, N = map(int, logits.shape)
-    dev = logits.device
+    if ws is not None:
+        _need(ws, "ws", torch.uint8)
+    dev = _on_device(logits, ws=ws)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     gates = torch.empty((T, k), dtype=torch.float32, device=dev)
     perm = torch.empty(T * k, dtype=torch.int32, device=dev)
@@ -216,11 +263,23 @@ def route(logits, k: int, ws=None, stream=None):
 def butterfly_apply(x, angles, expert_of_row=None, transpose: bool = False, ws=None, out=None, stream=None):
     """y[r] = B(angles[e_r]) x[r] (or B^T); x [rows][d] fp32/bf16 on the device."""
     torch = _torch()
+    _need(x, "x", dims=2)
+    _dt(x)
     rows, d = map(int, x.shape)
+    if not isinstance(angles, torch.Tensor) or angles.dim() < 1:
+        raise ValueError("angles must be a tensor [N][log2 d][d/2]")
     N = int(angles.shape[0])
+    _need(angles, "angles", torch.float32, numel=_angle_count(N, d))
+    if expert_of_row is not None:
+        _need(expert_of_row, "expert_of_row", torch.int32, numel=rows)
+    if out is not None:
+        _need(out, "out", x.dtype, numel=rows * d)
+    if ws is not None:
+        _need(ws, "ws", torch.uint8)
+    dev = _on_device(x, angles=angles, expert_of_row=expert_of_row, out=out, ws=ws)
     y = torch.empty_like(x) if out is None else out
     if ws is None:
-        ws = _ws(bfmoe_butterfly_workspace_bytes(d, N), x.device)
+        ws = _ws(bfmoe_butterfly_workspace_bytes(d, N), dev)
     _check(bfmoe_butterfly_apply(_ptr(x), _dt(x), rows, d, N, _ptr(angles), _ptr(expert_of_row),
                                  int(bool(transpose)), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
            "bfmoe_butterfly_apply")
@@ -231,14 +290,34 @@ def forward_workspace(T: int, d: int, N: int, k: int, device):
     return _ws(bfmoe_forward_workspace_bytes(T, d, N, k), device)
 
 
+def _check_layer_args(x, logits, packed, theta, phi, ws, out):
+    """Checks of forward's tensor arguments; returns (T, d, N, device)."""
+    torch = _torch()
+    _need(x, "x", dims=2)
+    _dt(x)
+    T, d = map(int, x.shape)
+    _need(logits, "logits", torch.float32, dims=2)
+    if int(logits.shape[0]) != T:
+        raise ValueError(f"logits has {int(logits.shape[0])} rows, x has {T}")
+    N = int(logits.shape[1])
+    _need(packed, "packed", torch.uint8, min_numel=int(bfmoe_packed_base_bytes(d)))
+    _need(theta, "theta", torch.float32, numel=_angle_count(N, d))
+    _need(phi, "phi", torch.float32, numel=_angle_count(N, d))
+    if out is not None:
+        _need(out, "out", x.dtype, numel=T * d)
+    if ws is not None:
+        _need(ws, "ws", torch.uint8)
+    dev = _on_device(x, logits=logits, packed=packed, theta=theta, phi=phi, out=out, ws=ws)
+    return T, d, N, dev
+
+
 def forward(x, logits, k: int, packed, theta, phi, ws=None, out=None, stream=None):
     """The expert layer: y = sum_j g_j alpha B(phi_e) W_base B(theta_e)^T x."""
     torch = _torch()
-    T, d = map(int, x.shape)
-    N = int(logits.shape[1])
+    T, d, N, dev = _check_layer_args(x, logits, packed, theta, phi, ws, out)
     y = torch.empty_like(x) if out is None else out
     if ws is None:
-        ws = forward_workspace(T, d, N, k, x.device)
+        ws = forward_workspace(T, d, N, k, dev)
     _check(bfmoe_forward(_ptr(x), _dt(x), T, d, _ptr(logits), N, k, _ptr(packed), _ptr(theta), _ptr(phi), _ptr(y),
                          _ptr(ws), ws.numel(), _stream(stream)), "bfmoe_forward")
     return y, ws
@@ -264,8 +343,7 @@ def forward_routing(ws, T: int, d: int, N: int, k: int):
 def forward_profile(x, logits, k: int, packed, theta, phi, ws, out, stream=None):
     """bfmoe_forward with a CUDA event after each kernel (synchronises);
     returns {stage name: milliseconds}."""
-    T, d = map(int, x.shape)
-    N = int(logits.shape[1])
+    T, d, N, _ = _check_layer_args(x, logits, packed, theta, phi, ws, out)
     ms = (ctypes.c_float * MAX_STAGES)()
     n = ctypes.c_int(0)
     _check(bfmoe_forward_profile(_ptr(x), _dt(x), T, d, _ptr(logits), N, k, _ptr(packed), _ptr(theta), _ptr(phi),
