@@ -36,6 +36,16 @@ MUTANTS = {
                            "return v == 1 ? 3u : (v == -1 ? 1u : 0u);"),
     "bucket_unstable": ("for (int i = 0; i < R; i++) perm[start[topk_idx[i]]++] = i;",
                         "for (int i = R - 1; i >= 0; i--) perm[start[topk_idx[i]]++] = i;"),
+    "gate_dropped_in_sum": ("yt[i] += g[(size_t)t * k + j] * u[i];", "yt[i] += u[i];"),
+    "offsets_inclusive": ("for (int e = 0; e <= N; e++) offsets[e] = start[e];",
+                          "for (int e = 0; e <= N; e++) offsets[e] = start[e < N ? e + 1 : N];"),
+    "zero_weight_as_plus_one": ("if (row[c] == 1) acc += x[c];", "if (row[c] >= 0) acc += x[c];"),
+    "nan_not_rejected": ("if (isnan(logits[i])) return ORACLE_ERR_NONFINITE;",
+                         "if (0 && isnan(logits[i])) return ORACLE_ERR_NONFINITE;"),
+    "pack_bit_order_reversed": ("word |= code_of(w[(size_t)r * d + 16 * wd + i]) << (2 * i);",
+                                "word |= code_of(w[(size_t)r * d + 16 * wd + i]) << (2 * (15 - i));"),
+    "all_minus_inf_gate": ("for (int j = 0; j < k; j++) g[j] = 1.0 / k;",
+                           "for (int j = 0; j < k; j++) g[j] = j == 0 ? 1.0 : 0.0;"),
 }
 
 
